@@ -1,0 +1,347 @@
+#!/usr/bin/env python3
+"""Benchmark of the fused chunked KL loss, forward + backward, on B200.
+
+One step = one fckl_fwd_bwd call over the whole workload (every chunk: teacher
+prep, fused projection + log-sum-exp, recompute + dlogits, dH and dW GEMMs).
+Default workload: the Llama-3.1-8B -> ~3B student shape at 8K context
+(N=8192, H=3072, V=128256, K=100, T=1, 5% rows masked).  Other configs are
+available with --config.
+
+Under torchrun with N ranks every rank runs its own replica of the workload on
+its own GPU (no data-path collective; "scaling": "weak"); the timing is the max
+over ranks.  `--impl reference` times the fp64 CPU oracle instead, on a bounded
+sample of rows of the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "fused KL fwd+bwd tokens/s & TFLOP/s (frac of BF16 peak); peak GiB vs seq len"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "source": "fallback"}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            d = json.load(fh)
+        d["source"] = "measured"
+        return d
+    except Exception:
+        return dict(FALLBACK_PEAKS)
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=0, help="rows in the oracle sample (0 = auto)")
+    ap.add_argument("--profile-json", default="")
+    return ap.parse_args()
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def workload_config(cfg: synth.Config, C: int) -> dict:
+    return {"workload": cfg.name, "N_rows": cfg.N, "H": cfg.H, "V": cfg.V, "K": cfg.K, "T": cfg.T,
+            "chunk": C, "mask_frac": cfg.mask_frac,
+            "l2": "inputs larger than L2 (W alone is %.0f MB > 126 MB)" % (cfg.V * cfg.H * 2 / 1e6),
+            "data": "synthetic seeded (synth recipe)"}
+
+
+# ------------------------------------------------------------------ oracle arm
+def oracle_rows_per_sec(inp, n_rows, reps=1):
+    import oracle
+    rows = synth.sample_rows(inp, n_rows)
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        oracle.oracle_from_inputs(inp, rows=rows, row_block=256)
+    dt = time.perf_counter() - t0
+    return rows.size * reps / dt, rows.size, dt
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def auto_cpu_rows(cfg):
+    # ~6*H*V fp64 flops per row; aim at ~10 s of host work at ~100 GFLOP/s
+    per_row = 6.0 * cfg.H * cfg.V
+    return int(max(16, min(1024, 1e12 / per_row)))
+
+
+def run_reference(args):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    cfg = synth.CONFIGS[args.config]
+    inp = synth.make_inputs(cfg)
+    n_rows = args.cpu_rows or max(8, auto_cpu_rows(cfg) // 8)
+    times = []
+    for i in range(args.warmup + args.steps):
+        rps, n, dt = oracle_rows_per_sec(inp, n_rows)
+        if i >= args.warmup:
+            times.append(dt)
+    ms = 1e3 * statistics.mean(times)
+    value = n_rows / (ms / 1e3)
+    sample = f"{n_rows} seeded valid rows of the workload per step (fwd + bwd incl. dW contribution)"
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": workload_config(cfg, 0),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_cores(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    def __init__(self, index):
+        self.proc = None
+        self.path = None
+        self.index = index
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as fh:
+            for ln in fh:
+                parts = [p.strip() for p in ln.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_cuda(args):
+    import torch
+    import torch.distributed as dist
+    from chunked_kl_loss_tcgen05_b200 import (FcklProblem, fckl_resolved_chunk,
+                                              fckl_profile_begin, fckl_profile_end)
+    from chunked_kl_loss_tcgen05_b200.torch_api import (alloc_workspace, arrays_to_device,
+                                                        fused_kl_fwd_bwd)
+
+    rank, local, world = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    cfg = synth.CONFIGS[args.config]
+    inp = synth.make_inputs(cfg)
+    prob = FcklProblem(cfg.N, cfg.H, cfg.V, cfg.K, cfg.T, cfg.chunk)
+    C = fckl_resolved_chunk(prob)
+    nchunks = -(-cfg.N // C)
+    launches_per_step = 2 + 6 * nchunks
+    n_valid = int(inp.row_mask.sum())
+    d = arrays_to_device(inp.hidden, inp.W, inp.topk_idx, inp.topk_logit, inp.row_mask, dev)
+    ws = alloc_workspace(prob, dev)
+    torch.cuda.synchronize()
+    torch.cuda.reset_peak_memory_stats(dev)
+
+    def step():
+        return fused_kl_fwd_bwd(*d, T=cfg.T, chunk=cfg.chunk, workspace=ws, check=False)
+
+    for _ in range(args.warmup):
+        out = step()
+    torch.cuda.synchronize()
+    from chunked_kl_loss_tcgen05_b200 import fckl_check
+    st = fckl_check(ws.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    if st != 0:
+        raise SystemExit(f"device error after warm-up: status {st}")
+    del out
+
+    clocks = ClockSampler(local)
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    fckl_profile_begin()
+    e0.record(stream)
+    for _ in range(args.steps):
+        out = step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    prof = fckl_profile_end()
+    clk = clocks.stop()
+    ms_total = e0.elapsed_time(e1)
+    peak_gib = torch.cuda.max_memory_allocated(dev) / 2**30
+    loss_val = float(out[0].item())
+    del out
+
+    t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    tokens = cfg.N * world
+    value = tokens / (ms_step / 1e3)
+    flops_step = 8.0 * cfg.H * cfg.V * n_valid
+    tflops = flops_step * world / (ms_step / 1e3) / 1e12
+
+    peaks = load_peaks()
+    # dominant kernel (largest share of the event-timed kernel time)
+    prof_total = sum(p["total_ms"] for p in prof) or 1.0
+    dom = max(prof, key=lambda p: p["total_ms"]) if prof else None
+    roofline = None
+    if dom is not None:
+        avg_ms = dom["total_ms"] / dom["launches"]
+        if dom["flops"] > 0:
+            peak = peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"]
+            ach = dom["flops"] / dom["launches"] / (avg_ms / 1e3) / 1e12
+            roofline = {"kernel": dom["name"], "bound": "tensor", "achieved": ach, "peak": peak,
+                        "unit": "TFLOP/s", "frac": ach / peak,
+                        "peak_kind": f"bf16_tflops_sustained ({peaks['source']})",
+                        "traffic": None, "share": dom["total_ms"] / prof_total}
+        else:
+            peak = peaks["hbm_gbs"]
+            ach = dom["bytes"] / dom["launches"] / (avg_ms / 1e3) / 1e9
+            roofline = {"kernel": dom["name"], "bound": "hbm", "achieved": ach, "peak": peak,
+                        "unit": "GB/s", "frac": ach / peak, "peak_kind": f"hbm_gbs ({peaks['source']})",
+                        "traffic": None, "share": dom["total_ms"] / prof_total}
+    kernels = [{"name": p["name"], "launches": p["launches"], "ms": p["total_ms"] / args.steps,
+                "share": p["total_ms"] / prof_total,
+                "tflops": (p["flops"] / (p["total_ms"] / 1e3) / 1e12) if p["flops"] else None}
+               for p in prof]
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = measure_e2e(torch, dev, inp, cfg, ws, max(3, min(args.steps, 5)), world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n_rows = args.cpu_rows or auto_cpu_rows(cfg)
+        rps, n, dt = oracle_rows_per_sec(inp, n_rows)
+        cpu = {"value": rps, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
+               "sample": f"{n} seeded valid rows of the workload, fwd+bwd incl. dW contribution, "
+                         f"{dt:.1f} s"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic",
+                "config": dict(workload_config(cfg, C), parallelism=f"replicas{world}",
+                               flush="inputs larger than L2"),
+                "tflops": tflops,
+                "frac_of_peak": {"measured_burst": tflops / world / peaks["bf16_tflops"],
+                                 "measured_sustained": tflops / world / peaks.get(
+                                     "bf16_tflops_sustained", peaks["bf16_tflops"]),
+                                 "dense_spec_2250": tflops / world / 2250.0},
+                "peak_mem_gib": peak_gib, "loss": loss_val,
+                "roofline": roofline, "kernels": kernels,
+                "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
+                "gpu_launches": launches_per_step * args.steps}
+        print(json.dumps(line), flush=True)
+        if args.profile_json:
+            with open(args.profile_json, "w") as fh:
+                json.dump(line, fh, indent=1)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def measure_e2e(torch, dev, inp, cfg, ws, steps, world):
+    """Same metric through the public API from pinned host buffers: every step
+    copies that step's inputs host->device and reads the loss back."""
+    from chunked_kl_loss_tcgen05_b200.torch_api import fused_kl_from_host
+    host = {"hidden": torch.from_numpy(inp.hidden.view(np.int16)).view(torch.bfloat16).pin_memory(),
+            "W": torch.from_numpy(inp.W.view(np.int16)).view(torch.bfloat16).pin_memory(),
+            "topk_idx": torch.from_numpy(inp.topk_idx).pin_memory(),
+            "topk_logit": torch.from_numpy(inp.topk_logit).pin_memory(),
+            "row_mask": torch.from_numpy(inp.row_mask).pin_memory()}
+    bufs = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    for _ in range(2):
+        fused_kl_from_host(bufs, host, T=cfg.T, chunk=cfg.chunk, workspace=ws)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fused_kl_from_host(bufs, host, T=cfg.T, chunk=cfg.chunk, workspace=ws)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    del bufs
+    return {"value": cfg.N * world / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": 4, "steps": steps}
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_cuda(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,149 @@
+"""Fused chunked forward-KL distillation loss on B200 (sm_100a).
+
+Thin ctypes binding over the C ABI in ``include/fckl.h`` (``libfckl.so``, built
+in-tree by ``chunked_kl_loss_tcgen05_b200.build``).  The functions below keep
+the C names and only marshal arguments; every step of the loss runs in the
+library's CUDA kernels.  There is no CPU fallback: if the library is missing,
+``load()`` raises.
+
+``torch_api`` adds tensor-level helpers (allocation of outputs and workspace
+with PyTorch, an autograd Function) on top of these calls.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "FCKL_OK", "FCKL_ERR_INVALID_ARG", "FCKL_ERR_UNSUPPORTED", "FCKL_ERR_WORKSPACE",
+    "FCKL_ERR_BAD_INDEX", "FCKL_ERR_BAD_TEACHER", "FCKL_ERR_TIMEOUT", "FCKL_ERR_CUDA",
+    "FCKL_K_MAX", "FcklProblem", "FcklError", "load", "lib_path", "exported_symbols",
+    "fckl_workspace_bytes", "fckl_resolved_chunk", "fckl_fwd", "fckl_fwd_bwd", "fckl_check",
+    "fckl_status_string", "FcklKernelStat", "fckl_profile_begin", "fckl_profile_end",
+]
+
+FCKL_OK = 0
+FCKL_ERR_INVALID_ARG = 1
+FCKL_ERR_UNSUPPORTED = 2
+FCKL_ERR_WORKSPACE = 3
+FCKL_ERR_BAD_INDEX = 4
+FCKL_ERR_BAD_TEACHER = 5
+FCKL_ERR_TIMEOUT = 6
+FCKL_ERR_CUDA = 7
+FCKL_K_MAX = 256
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB = None
+
+exported_symbols = ("fckl_workspace_bytes", "fckl_resolved_chunk", "fckl_fwd", "fckl_fwd_bwd",
+                    "fckl_check", "fckl_status_string", "fckl_profile_begin", "fckl_profile_end")
+
+
+class FcklProblem(ctypes.Structure):
+    """Mirror of ``fckl_problem``."""
+    _fields_ = [("N", ctypes.c_int64), ("H", ctypes.c_int64), ("V", ctypes.c_int64),
+                ("K", ctypes.c_int32), ("T", ctypes.c_float), ("chunk", ctypes.c_int64)]
+
+    def __init__(self, N, H, V, K, T=1.0, chunk=0):
+        super().__init__(int(N), int(H), int(V), int(K), float(T), int(chunk))
+
+
+class FcklKernelStat(ctypes.Structure):
+    """Mirror of ``fckl_kernel_stat``."""
+    _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int64),
+                ("total_ms", ctypes.c_double), ("flops", ctypes.c_double),
+                ("bytes", ctypes.c_double)]
+
+
+class FcklError(RuntimeError):
+    def __init__(self, status: int, where: str = ""):
+        self.status = int(status)
+        super().__init__(f"{where}: {fckl_status_string(status)} ({status})")
+
+
+def lib_path() -> str:
+    return os.environ.get("FCKL_LIB", os.path.join(_HERE, "libfckl.so"))
+
+
+def load() -> ctypes.CDLL:
+    """Load libfckl.so (raises if it has not been built)."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    path = lib_path()
+    if not os.path.exists(path):
+        raise FileNotFoundError(
+            f"{path} is missing; build it with `python -m chunked_kl_loss_tcgen05_b200.build`")
+    lib = ctypes.CDLL(path)
+    P = ctypes.POINTER(FcklProblem)
+    vp, sz = ctypes.c_void_p, ctypes.c_size_t
+    lib.fckl_workspace_bytes.argtypes = [P]
+    lib.fckl_workspace_bytes.restype = sz
+    lib.fckl_resolved_chunk.argtypes = [P]
+    lib.fckl_resolved_chunk.restype = ctypes.c_int64
+    lib.fckl_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.fckl_fwd.restype = ctypes.c_int
+    lib.fckl_fwd_bwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.fckl_fwd_bwd.restype = ctypes.c_int
+    lib.fckl_check.argtypes = [vp, vp]
+    lib.fckl_check.restype = ctypes.c_int
+    lib.fckl_status_string.argtypes = [ctypes.c_int]
+    lib.fckl_status_string.restype = ctypes.c_char_p
+    lib.fckl_profile_begin.argtypes = []
+    lib.fckl_profile_begin.restype = None
+    lib.fckl_profile_end.argtypes = [ctypes.POINTER(FcklKernelStat), ctypes.c_int]
+    lib.fckl_profile_end.restype = ctypes.c_int
+    _LIB = lib
+    return lib
+
+
+def _ptr(x):
+    return None if x is None or x == 0 else ctypes.c_void_p(int(x))
+
+
+def fckl_workspace_bytes(prob: FcklProblem) -> int:
+    return int(load().fckl_workspace_bytes(ctypes.byref(prob)))
+
+
+def fckl_resolved_chunk(prob: FcklProblem) -> int:
+    return int(load().fckl_resolved_chunk(ctypes.byref(prob)))
+
+
+def fckl_fwd(prob, hidden, W, topk_idx, topk_logit, row_mask, loss, row_loss,
+             workspace, workspace_bytes, stream) -> int:
+    """All array arguments are device addresses (ints) or None; returns the status."""
+    return int(load().fckl_fwd(ctypes.byref(prob), _ptr(hidden), _ptr(W), _ptr(topk_idx),
+                               _ptr(topk_logit), _ptr(row_mask), _ptr(loss), _ptr(row_loss),
+                               _ptr(workspace), ctypes.c_size_t(int(workspace_bytes)),
+                               _ptr(stream)))
+
+
+def fckl_fwd_bwd(prob, hidden, W, topk_idx, topk_logit, row_mask, loss, row_loss, dH, dW,
+                 workspace, workspace_bytes, stream) -> int:
+    """All array arguments are device addresses (ints) or None; returns the status."""
+    return int(load().fckl_fwd_bwd(ctypes.byref(prob), _ptr(hidden), _ptr(W), _ptr(topk_idx),
+                                   _ptr(topk_logit), _ptr(row_mask), _ptr(loss),
+                                   _ptr(row_loss), _ptr(dH), _ptr(dW), _ptr(workspace),
+                                   ctypes.c_size_t(int(workspace_bytes)), _ptr(stream)))
+
+
+def fckl_check(workspace, stream) -> int:
+    return int(load().fckl_check(_ptr(workspace), _ptr(stream)))
+
+
+def fckl_status_string(status: int) -> str:
+    return load().fckl_status_string(int(status)).decode()
+
+
+def fckl_profile_begin() -> None:
+    load().fckl_profile_begin()
+
+
+def fckl_profile_end(max_stats: int = 16) -> list:
+    """Returns a list of dicts (name, launches, total_ms, flops, bytes)."""
+    arr = (FcklKernelStat * max_stats)()
+    n = int(load().fckl_profile_end(arr, max_stats))
+    if n < 0:
+        raise FcklError(FCKL_ERR_CUDA, "fckl_profile_end")
+    return [dict(name=a.name.decode(), launches=int(a.launches), total_ms=float(a.total_ms),
+                 flops=float(a.flops), bytes=float(a.bytes)) for a in arr[:min(n, max_stats)]]

@@ -1,0 +1,472 @@
+// Host side of libfckl: argument checks, workspace layout, tensor maps and the
+// chunk scheduler that enqueues the kernels of every chunk on the caller's
+// stream.  The library allocates no memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "fckl.h"
+#include "epilogues.cuh"
+#include "gemm.cuh"
+#include "ptx.cuh"
+#include "rows.cuh"
+
+using namespace fckl;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr int kMaxDevices = 64;
+constexpr int kMaxGrid = 1024;  // partial-statistics slots are sized for at most this many CTAs
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
+
+struct Layout {
+  long long N, H, V, K, C, Vp, nchunks, RBmax;
+  size_t off_rowloss, off_sid, off_sp, off_zs, off_plogp, off_lse2, off_part, off_dlog, total;
+  size_t part_slots;  // float2 entries reserved for partial statistics
+};
+
+bool valid_problem(const fckl_problem* p) {
+  if (p == nullptr) return false;
+  if (p->N < 1 || p->H < 1 || p->V < 1 || p->K < 1 || p->chunk < 0) return false;
+  if (!(std::isfinite(p->T) && p->T > 0.f)) return false;
+  if (p->N > INT32_MAX || p->H > INT32_MAX || p->V > INT32_MAX) return false;
+  return true;
+}
+
+bool supported_problem(const fckl_problem* p) {
+  return p->K <= FCKL_K_MAX && p->K <= p->V && p->H % 8 == 0;
+}
+
+long long resolve_chunk(const fckl_problem* p) {
+  const long long Vp = align_up((size_t)p->V, 8);
+  long long C = p->chunk;
+  if (C == 0) {
+    const long long budget = 512ll << 20;
+    C = budget / (Vp * 2) / 128 * 128;
+    C = std::max(C, 128ll);
+    C = std::min(C, (long long)align_up((size_t)p->N, 64));
+  }
+  return std::min<long long>(C, p->N);
+}
+
+Layout make_layout(const fckl_problem* p) {
+  Layout L{};
+  L.N = p->N; L.H = p->H; L.V = p->V; L.K = p->K;
+  L.Vp = (long long)align_up((size_t)p->V, 8);
+  L.C = resolve_chunk(p);
+  L.nchunks = cdiv(L.N, L.C);
+  L.RBmax = cdiv(L.C, BM);
+  size_t off = align_up(sizeof(DeviceCtl), kAlign);
+  auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, kAlign); return o; };
+  L.off_rowloss = take((size_t)L.N * 4);
+  L.off_sid = take((size_t)L.C * L.K * 4);
+  L.off_sp = take((size_t)L.C * L.K * 4);
+  L.off_zs = take((size_t)L.C * L.K * 4);
+  L.off_plogp = take((size_t)L.C * 4);
+  L.off_lse2 = take((size_t)L.C * 4);
+  L.part_slots = (size_t)(kMaxGrid + 2 * L.RBmax) * BM;
+  L.off_part = take(L.part_slots * sizeof(float2));
+  L.off_dlog = take((size_t)L.C * L.Vp * 2);
+  L.total = off;
+  return L;
+}
+
+// ---------------------------------------------------------------- tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// bf16 2-D map: inner (contiguous) extent, outer extent, outer stride in bytes,
+// box {box_inner, box_outer}, 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap* m, const void* base, long long inner, long long outer,
+              long long stride_bytes, int box_inner, int box_outer) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+  cuuint64_t strides[1] = {(cuuint64_t)stride_bytes};
+  cuuint32_t box[2] = {(cuuint32_t)box_inner, (cuuint32_t)box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- device info
+struct DeviceInfo {
+  bool ready = false;
+  bool ok = false;
+  int sms = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+template <class Sched, class Epi, bool A_MN, bool B_MN>
+bool set_smem_attr() {
+  return cudaFuncSetAttribute(gemm_kernel<Sched, Epi, A_MN, B_MN>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)GEMM_SMEM_BYTES) == cudaSuccess;
+}
+
+const DeviceInfo* device_info() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    d.ready = true;
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+    d.ok = major == 10 && minor == 0 && d.sms > 0;
+    if (d.ok) {
+      d.ok = set_smem_attr<SchedLinear, EpiLse, false, false>() &&
+             set_smem_attr<SchedLinear, EpiDlogits, false, false>() &&
+             set_smem_attr<SchedSplitK, EpiDH, false, true>() &&
+             set_smem_attr<SchedTiles, EpiDW, true, true>();
+    }
+    d.sms = std::min(d.sms, kMaxGrid);
+  }
+  return &d;
+}
+
+// ---------------------------------------------------------------- knobs
+uint64_t wait_timeout_ns() {
+  const char* s = std::getenv("FCKL_WAIT_TIMEOUT_MS");
+  long long ms = s ? std::atoll(s) : 2000;
+  if (ms < 1) ms = 1;
+  if (ms > 60000) ms = 60000;
+  return (uint64_t)ms * 1000000ull;
+}
+int debug_skip_commit() {
+  const char* s = std::getenv("FCKL_DEBUG_SKIP_ARRIVE");
+  return (s && std::atoi(s) > 0) ? 1 : 0;
+}
+
+// ---------------------------------------------------------------- profiling
+enum Kind { K_COUNT, K_PREP, K_FWD, K_MERGE, K_BWD, K_DH, K_DW, K_FINAL, K_NKINDS };
+const char* const kKindName[K_NKINDS] = {"count_valid", "prep_teacher", "fwd_logits_lse",
+                                         "merge_loss", "bwd_dlogits", "dH_gemm", "dW_gemm",
+                                         "finalize"};
+struct ProfRec {
+  int kind;
+  cudaEvent_t a, b;
+  double flops, bytes;
+};
+struct Profiler {
+  bool on = false;
+  std::vector<ProfRec> recs;
+  std::vector<cudaEvent_t> pool;
+  size_t used = 0;
+  cudaEvent_t next() {
+    if (used == pool.size()) {
+      cudaEvent_t e = nullptr;
+      if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+      pool.push_back(e);
+    }
+    return pool[used++];
+  }
+};
+Profiler g_prof;
+
+struct ProfScope {
+  int kind;
+  cudaStream_t st;
+  double flops, bytes;
+  cudaEvent_t a = nullptr;
+  ProfScope(int k, cudaStream_t s, double f, double b) : kind(k), st(s), flops(f), bytes(b) {
+    if (g_prof.on && (a = g_prof.next()) != nullptr) cudaEventRecord(a, st);
+  }
+  ~ProfScope() {
+    if (!g_prof.on || a == nullptr) return;
+    cudaEvent_t b = g_prof.next();
+    if (b == nullptr) return;
+    cudaEventRecord(b, st);
+    g_prof.recs.push_back(ProfRec{kind, a, b, flops, bytes});
+  }
+};
+
+// Split-K factor for dH: minimise waves * (k-blocks per unit + fixed cost).
+int choose_split(long long tiles, long long KB, int sms) {
+  int best = 1;
+  double best_cost = 1e300;
+  const long long smax = std::min<long long>(KB, 512);
+  for (long long S = 1; S <= smax; ++S) {
+    const long long units = tiles * S;
+    const double waves = (double)cdiv(units, sms);
+    const double cost = waves * ((double)cdiv(KB, S) + 6.0);
+    if (cost < best_cost - 1e-9) { best_cost = cost; best = (int)S; }
+  }
+  return best;
+}
+
+int max_splits(long long RB, long long NT, long long total, long long G) {
+  long long m = 1;
+  for (long long rb = 0; rb < RB; ++rb) {
+    const long long n = lin_owner(rb * NT + NT - 1, total, G) - lin_owner(rb * NT, total, G) + 1;
+    m = std::max(m, n);
+  }
+  return (int)m;
+}
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+fckl_status run(bool bwd, const fckl_problem* prob, const void* hidden, const void* W,
+                const int32_t* topk_idx, const float* topk_logit, const uint8_t* row_mask,
+                float* loss, float* row_loss, float* dH, float* dW, void* workspace,
+                size_t ws_bytes, void* stream_ptr) {
+  if (!valid_problem(prob)) return FCKL_ERR_INVALID_ARG;
+  if (!hidden || !W || !topk_idx || !topk_logit || !loss) return FCKL_ERR_INVALID_ARG;
+  if (bwd && (!dH || !dW)) return FCKL_ERR_INVALID_ARG;
+  if (!aligned(hidden, 16) || !aligned(W, 16) || !aligned(topk_idx, 4) ||
+      !aligned(topk_logit, 4) || !aligned(loss, 4) || (row_loss && !aligned(row_loss, 4)) ||
+      (bwd && (!aligned(dH, 16) || !aligned(dW, 16))))
+    return FCKL_ERR_INVALID_ARG;
+  if (!supported_problem(prob)) return FCKL_ERR_UNSUPPORTED;
+  const Layout L = make_layout(prob);
+  if (workspace == nullptr || !aligned(workspace, kAlign) || ws_bytes < L.total)
+    return FCKL_ERR_WORKSPACE;
+  const DeviceInfo* dev = device_info();
+  if (dev == nullptr || !dev->ok) return FCKL_ERR_UNSUPPORTED;
+  if (get_encode_fn() == nullptr) return FCKL_ERR_CUDA;
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_ptr);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  DeviceCtl* ctl = reinterpret_cast<DeviceCtl*>(ws);
+  float* rl = row_loss ? row_loss : reinterpret_cast<float*>(ws + L.off_rowloss);
+  int* sid = reinterpret_cast<int*>(ws + L.off_sid);
+  float* sp = reinterpret_cast<float*>(ws + L.off_sp);
+  float* zs = reinterpret_cast<float*>(ws + L.off_zs);
+  float* plogp = reinterpret_cast<float*>(ws + L.off_plogp);
+  float* lse2 = reinterpret_cast<float*>(ws + L.off_lse2);
+  float2* part = reinterpret_cast<float2*>(ws + L.off_part);
+  __nv_bfloat16* dlog = reinterpret_cast<__nv_bfloat16*>(ws + L.off_dlog);
+
+  const int H = (int)L.H, V = (int)L.V, K = (int)L.K;
+  const float invT = 1.0f / prob->T;
+  const float scale2 = 1.4426950408889634f / prob->T;
+  CtlArgs ca{ctl, wait_timeout_ns(), debug_skip_commit()};
+
+  if (cudaMemsetAsync(ctl, 0, sizeof(DeviceCtl), st) != cudaSuccess) return FCKL_ERR_CUDA;
+  {
+    ProfScope ps(K_COUNT, st, 0.0, row_mask ? (double)L.N : 0.0);
+    k_count_valid<<<1, 1024, 0, st>>>(row_mask, L.N, ctl);
+  }
+
+  CUtensorMap mapW_k, mapW_mn;
+  if (!make_map(&mapW_k, W, L.H, L.V, L.H * 2, BK, BN)) return FCKL_ERR_CUDA;
+  if (bwd && !make_map(&mapW_mn, W, L.H, L.V, L.H * 2, 64, BK)) return FCKL_ERR_CUDA;
+
+  const long long NT = cdiv(L.V, BN);
+  const long long KBh = cdiv(L.H, BK);
+  for (long long c = 0; c < L.nchunks; ++c) {
+    const long long row0 = c * L.C;
+    const int rows = (int)std::min(L.C, L.N - row0);
+    const long long RB = cdiv(rows, BM);
+    const uint8_t* mask_c = row_mask ? row_mask + row0 : nullptr;
+    const void* h_c = static_cast<const uint8_t*>(hidden) + (size_t)row0 * L.H * 2;
+    const int row_blocks = (int)cdiv(rows, ROW_WARPS);
+
+    {
+      ProfScope ps(K_PREP, st, 0.0, (double)rows * K * 20.0 + rows * 5.0);
+      k_prep_teacher<<<row_blocks, ROW_WARPS * 32, 0, st>>>(
+          topk_idx + row0 * K, topk_logit + row0 * K, mask_c, rows, K, V, invT, sid, sp, zs,
+          plogp, ctl);
+    }
+
+    CUtensorMap mapH_k;
+    if (!make_map(&mapH_k, h_c, L.H, rows, L.H * 2, BK, BM)) return FCKL_ERR_CUDA;
+
+    const long long total = RB * NT;
+    const int G = (int)std::min<long long>(dev->sms, total);
+    const int Smax = max_splits(RB, NT, total, G);
+    if ((size_t)RB * Smax * BM > L.part_slots) return FCKL_ERR_UNSUPPORTED;
+    SchedArgs sa_lin{total, (int)NT, (int)KBh, 1, 0};
+
+    EpiLse::Params pf{rows, V, K, Smax, scale2, sid, zs, part};
+    CtlArgs ca_f = ca;
+    ca_f.debug_skip_commit = (c == 0) ? ca.debug_skip_commit : 0;
+    const double gemm_flops = 2.0 * rows * (double)L.V * (double)L.H;
+    {
+      ProfScope ps(K_FWD, st, gemm_flops, 2.0 * (rows + (double)L.V) * L.H + rows * K * 4.0);
+      gemm_kernel<SchedLinear, EpiLse, false, false>
+          <<<G, GEMM_THREADS, GEMM_SMEM_BYTES, st>>>(mapH_k, mapW_k, pf, sa_lin, ca_f);
+    }
+
+    {
+      ProfScope ps(K_MERGE, st, 0.0, (double)rows * K * 8.0 + rows * 13.0);
+      k_merge_loss<<<row_blocks, ROW_WARPS * 32, 0, st>>>(part, Smax, (int)NT, total, G, rows,
+                                                           K, invT, zs, sp, plogp, mask_c, lse2,
+                                                           rl + row0);
+    }
+    if (!bwd) continue;
+
+    EpiDlogits::Params pb{rows, V, (int)L.Vp, K, scale2, lse2, sid, sp, mask_c, dlog};
+    {
+      ProfScope ps(K_BWD, st, gemm_flops, 2.0 * (rows + (double)L.V) * L.H + 2.0 * rows * L.Vp);
+      gemm_kernel<SchedLinear, EpiDlogits, false, false>
+          <<<G, GEMM_THREADS, GEMM_SMEM_BYTES, st>>>(mapH_k, mapW_k, pb, sa_lin, ca);
+    }
+
+    // dH[rows] = alpha * dlogits W : A = dlogits (K-major), B = W (MN-major).
+    if (cudaMemsetAsync(dH + row0 * L.H, 0, (size_t)rows * L.H * 4, st) != cudaSuccess)
+      return FCKL_ERR_CUDA;
+    CUtensorMap mapD_k, mapD_mn, mapH_mn;
+    if (!make_map(&mapD_k, dlog, L.V, rows, L.Vp * 2, BK, BM)) return FCKL_ERR_CUDA;
+    const long long NTh = cdiv(L.H, BN);
+    const long long tiles_h = RB * NTh;
+    const long long KBv = cdiv(L.V, BK);
+    const int S = choose_split(tiles_h, KBv, dev->sms);
+    SchedArgs sa_dh{tiles_h * S, (int)NTh, (int)KBv, S, (int)tiles_h};
+    const int Gh = (int)std::min<long long>(dev->sms, tiles_h * S);
+    EpiDH::Params ph{rows, H, invT, ctl, dH + row0 * L.H};
+    {
+      ProfScope ps(K_DH, st, gemm_flops,
+                   2.0 * rows * (double)L.V + 2.0 * (double)L.V * L.H + 4.0 * rows * L.H);
+      gemm_kernel<SchedSplitK, EpiDH, false, true>
+          <<<Gh, GEMM_THREADS, GEMM_SMEM_BYTES, st>>>(mapD_k, mapW_mn, ph, sa_dh, ca);
+    }
+
+    // dW (+)= alpha * dlogits^T h : A = dlogits^T (MN-major), B = h (MN-major).
+    if (!make_map(&mapD_mn, dlog, L.V, rows, L.Vp * 2, 64, BK)) return FCKL_ERR_CUDA;
+    if (!make_map(&mapH_mn, h_c, L.H, rows, L.H * 2, 64, BK)) return FCKL_ERR_CUDA;
+    const long long tiles_w = cdiv(L.V, BM) * NTh;
+    SchedArgs sa_dw{tiles_w, (int)NTh, (int)cdiv(rows, BK), 1, (int)tiles_w};
+    const int Gw = (int)std::min<long long>(dev->sms, tiles_w);
+    EpiDW::Params pw{V, H, invT, c > 0 ? 1 : 0, ctl, dW};
+    {
+      ProfScope ps(K_DW, st, gemm_flops,
+                   2.0 * rows * (double)L.V + 2.0 * rows * L.H +
+                       (c > 0 ? 8.0 : 4.0) * (double)L.V * L.H);
+      gemm_kernel<SchedTiles, EpiDW, true, true>
+          <<<Gw, GEMM_THREADS, GEMM_SMEM_BYTES, st>>>(mapD_mn, mapH_mn, pw, sa_dw, ca);
+    }
+  }
+  {
+    ProfScope ps(K_FINAL, st, 0.0, (double)L.N * 4.0);
+    k_finalize<<<1, 1024, 0, st>>>(rl, L.N, ctl, loss);
+  }
+  if (cudaGetLastError() != cudaSuccess) return FCKL_ERR_CUDA;
+  return FCKL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t fckl_workspace_bytes(const fckl_problem* prob) {
+  if (!valid_problem(prob) || !supported_problem(prob)) return 0;
+  return make_layout(prob).total;
+}
+
+int64_t fckl_resolved_chunk(const fckl_problem* prob) {
+  if (!valid_problem(prob) || !supported_problem(prob)) return -1;
+  return resolve_chunk(prob);
+}
+
+fckl_status fckl_fwd(const fckl_problem* prob, const void* hidden, const void* W,
+                     const int32_t* topk_idx, const float* topk_logit, const uint8_t* row_mask,
+                     float* loss, float* row_loss, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+  return run(false, prob, hidden, W, topk_idx, topk_logit, row_mask, loss, row_loss, nullptr,
+             nullptr, workspace, workspace_bytes, stream);
+}
+
+fckl_status fckl_fwd_bwd(const fckl_problem* prob, const void* hidden, const void* W,
+                         const int32_t* topk_idx, const float* topk_logit,
+                         const uint8_t* row_mask, float* loss, float* row_loss, float* dH,
+                         float* dW, void* workspace, size_t workspace_bytes, void* stream) {
+  return run(true, prob, hidden, W, topk_idx, topk_logit, row_mask, loss, row_loss, dH, dW,
+             workspace, workspace_bytes, stream);
+}
+
+fckl_status fckl_check(void* workspace, void* stream) {
+  if (workspace == nullptr) return FCKL_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t err = 0;
+  if (cudaMemcpyAsync(&err, workspace, sizeof(err), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return FCKL_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return FCKL_ERR_CUDA;
+  if (err & kErrTimeout) return FCKL_ERR_TIMEOUT;
+  if (err & kErrBadIndex) return FCKL_ERR_BAD_INDEX;
+  if (err & kErrBadTeacher) return FCKL_ERR_BAD_TEACHER;
+  return FCKL_OK;
+}
+
+void fckl_profile_begin(void) {
+  g_prof.on = true;
+  g_prof.recs.clear();
+  g_prof.used = 0;
+}
+
+int fckl_profile_end(fckl_kernel_stat* stats, int max_stats) {
+  g_prof.on = false;
+  int order[K_NKINDS];
+  int nkinds = 0;
+  fckl_kernel_stat acc[K_NKINDS];
+  std::memset(acc, 0, sizeof(acc));
+  int slot[K_NKINDS];
+  for (int k = 0; k < K_NKINDS; ++k) slot[k] = -1;
+  for (const ProfRec& r : g_prof.recs) {
+    if (cudaEventSynchronize(r.b) != cudaSuccess) return -1;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) return -1;
+    if (slot[r.kind] < 0) {
+      slot[r.kind] = nkinds;
+      order[nkinds++] = r.kind;
+    }
+    fckl_kernel_stat& a = acc[slot[r.kind]];
+    a.launches += 1;
+    a.total_ms += ms;
+    a.flops += r.flops;
+    a.bytes += r.bytes;
+  }
+  for (int i = 0; i < nkinds && i < max_stats && stats; ++i) {
+    stats[i] = acc[i];
+    std::strncpy(stats[i].name, kKindName[order[i]], sizeof(stats[i].name) - 1);
+    stats[i].name[sizeof(stats[i].name) - 1] = 0;
+  }
+  g_prof.recs.clear();
+  g_prof.used = 0;
+  return nkinds;
+}
+
+const char* fckl_status_string(fckl_status s) {
+  switch (s) {
+    case FCKL_OK: return "FCKL_OK";
+    case FCKL_ERR_INVALID_ARG: return "FCKL_ERR_INVALID_ARG";
+    case FCKL_ERR_UNSUPPORTED: return "FCKL_ERR_UNSUPPORTED";
+    case FCKL_ERR_WORKSPACE: return "FCKL_ERR_WORKSPACE";
+    case FCKL_ERR_BAD_INDEX: return "FCKL_ERR_BAD_INDEX";
+    case FCKL_ERR_BAD_TEACHER: return "FCKL_ERR_BAD_TEACHER";
+    case FCKL_ERR_TIMEOUT: return "FCKL_ERR_TIMEOUT";
+    case FCKL_ERR_CUDA: return "FCKL_ERR_CUDA";
+  }
+  return "FCKL_ERR_UNKNOWN";
+}
+
+}  // extern "C"

@@ -1,0 +1,157 @@
+"""Tensor-level helpers over the C ABI (PyTorch supplies memory and streams only).
+
+``fused_kl_fwd_bwd`` / ``fused_kl_fwd`` allocate outputs and the workspace
+with PyTorch on the inputs' device and call the library on the current
+stream.  ``FusedChunkedKL`` is an autograd Function that computes the
+gradients inside its forward (one fused library call) and scales them by the
+upstream gradient in backward.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import (FcklError, FcklProblem, FCKL_OK, fckl_check, fckl_fwd, fckl_fwd_bwd,
+               fckl_workspace_bytes)
+
+__all__ = ["make_problem", "alloc_workspace", "fused_kl_fwd", "fused_kl_fwd_bwd",
+           "fused_kl_from_host", "FusedChunkedKL", "fused_chunked_kl_loss"]
+
+
+def _bits(t: torch.Tensor) -> torch.Tensor:
+    if t.dtype == torch.bfloat16:
+        return t
+    if t.dtype in (torch.int16, torch.uint16):
+        return t.view(torch.bfloat16)
+    raise TypeError(f"expected bfloat16 (or its uint16 bits), got {t.dtype}")
+
+
+def make_problem(hidden, W, topk_idx, T=1.0, chunk=0) -> FcklProblem:
+    N, H = hidden.shape
+    V = W.shape[0]
+    K = topk_idx.shape[1]
+    return FcklProblem(N, H, V, K, T, chunk)
+
+
+def alloc_workspace(prob: FcklProblem, device) -> torch.Tensor:
+    nbytes = fckl_workspace_bytes(prob)
+    if nbytes == 0:
+        raise FcklError(1, "fckl_workspace_bytes")
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def _check_inputs(hidden, W, topk_idx, topk_logit, row_mask):
+    for name, t in (("hidden", hidden), ("W", W), ("topk_idx", topk_idx),
+                    ("topk_logit", topk_logit)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if topk_idx.dtype != torch.int32 or topk_logit.dtype != torch.float32:
+        raise TypeError("topk_idx must be int32 and topk_logit float32")
+    if row_mask is not None and (row_mask.dtype != torch.uint8 or not row_mask.is_contiguous()):
+        raise TypeError("row_mask must be a contiguous uint8 tensor")
+
+
+def fused_kl_fwd_bwd(hidden, W, topk_idx, topk_logit, row_mask=None, T=1.0, chunk=0,
+                     workspace=None, want_row_loss=False, check=True):
+    """Returns (loss[1], row_loss[N] or None, dH[N,H] fp32, dW[V,H] fp32)."""
+    hidden, W = _bits(hidden), _bits(W)
+    _check_inputs(hidden, W, topk_idx, topk_logit, row_mask)
+    prob = make_problem(hidden, W, topk_idx, T, chunk)
+    dev = hidden.device
+    if workspace is None:
+        workspace = alloc_workspace(prob, dev)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    row_loss = torch.empty(prob.N, dtype=torch.float32, device=dev) if want_row_loss else None
+    dH = torch.empty(prob.N, prob.H, dtype=torch.float32, device=dev)
+    dW = torch.empty(prob.V, prob.H, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    st = fckl_fwd_bwd(prob, hidden.data_ptr(), W.data_ptr(), topk_idx.data_ptr(),
+                      topk_logit.data_ptr(), None if row_mask is None else row_mask.data_ptr(),
+                      loss.data_ptr(), None if row_loss is None else row_loss.data_ptr(),
+                      dH.data_ptr(), dW.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                      stream)
+    if st != FCKL_OK:
+        raise FcklError(st, "fckl_fwd_bwd")
+    if check:
+        st = fckl_check(workspace.data_ptr(), stream)
+        if st != FCKL_OK:
+            raise FcklError(st, "fckl_check")
+    return loss, row_loss, dH, dW
+
+
+def fused_kl_fwd(hidden, W, topk_idx, topk_logit, row_mask=None, T=1.0, chunk=0,
+                 workspace=None, want_row_loss=False, check=True):
+    """Returns (loss[1], row_loss[N] or None)."""
+    hidden, W = _bits(hidden), _bits(W)
+    _check_inputs(hidden, W, topk_idx, topk_logit, row_mask)
+    prob = make_problem(hidden, W, topk_idx, T, chunk)
+    dev = hidden.device
+    if workspace is None:
+        workspace = alloc_workspace(prob, dev)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    row_loss = torch.empty(prob.N, dtype=torch.float32, device=dev) if want_row_loss else None
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    st = fckl_fwd(prob, hidden.data_ptr(), W.data_ptr(), topk_idx.data_ptr(),
+                  topk_logit.data_ptr(), None if row_mask is None else row_mask.data_ptr(),
+                  loss.data_ptr(), None if row_loss is None else row_loss.data_ptr(),
+                  workspace.data_ptr(), workspace.numel(), stream)
+    if st != FCKL_OK:
+        raise FcklError(st, "fckl_fwd")
+    if check:
+        st = fckl_check(workspace.data_ptr(), stream)
+        if st != FCKL_OK:
+            raise FcklError(st, "fckl_check")
+    return loss, row_loss
+
+
+def fused_kl_from_host(dev_bufs: dict, host: dict, T=1.0, chunk=0, workspace=None):
+    """End-to-end call from pinned host arrays: copies the inputs host->device on
+    the current stream, runs fused forward+backward, and reads the loss back.
+    ``dev_bufs`` holds preallocated device tensors with the same keys as
+    ``host`` (hidden, W, topk_idx, topk_logit, row_mask).  Returns (loss as a
+    Python float, dH, dW)."""
+    for k, h in host.items():
+        dev_bufs[k].copy_(h, non_blocking=True)
+    loss, _, dH, dW = fused_kl_fwd_bwd(dev_bufs["hidden"], dev_bufs["W"], dev_bufs["topk_idx"],
+                                       dev_bufs["topk_logit"], dev_bufs.get("row_mask"), T=T,
+                                       chunk=chunk, workspace=workspace, check=False)
+    return float(loss.item()), dH, dW
+
+
+class FusedChunkedKL(torch.autograd.Function):
+    """loss = FusedChunkedKL.apply(hidden_bf16, W_bf16, topk_idx, topk_logit, row_mask, T, chunk)
+
+    Gradients flow to hidden and W (returned as fp32 tensors cast to the input
+    dtype); the fused call computes them in forward."""
+
+    @staticmethod
+    def forward(ctx, hidden, W, topk_idx, topk_logit, row_mask, T, chunk):
+        loss, _, dH, dW = fused_kl_fwd_bwd(hidden, W, topk_idx, topk_logit, row_mask, T, chunk)
+        ctx.save_for_backward(dH, dW)
+        ctx.dtypes = (hidden.dtype, W.dtype)
+        return loss[0]
+
+    @staticmethod
+    def backward(ctx, grad_out):
+        dH, dW = ctx.saved_tensors
+        return ((dH * grad_out).to(ctx.dtypes[0]), (dW * grad_out).to(ctx.dtypes[1]),
+                None, None, None, None, None)
+
+
+def fused_chunked_kl_loss(hidden, W, topk_idx, topk_logit, row_mask=None, T=1.0, chunk=0):
+    return FusedChunkedKL.apply(hidden, W, topk_idx, topk_logit, row_mask, T, chunk)
+
+
+def arrays_to_device(hidden_bits, W_bits, topk_idx, topk_logit, row_mask, device="cuda"):
+    """numpy arrays (bf16 bit patterns as uint16, int32 ids, float32 logits,
+    uint8 mask or None) -> contiguous device tensors, in that order."""
+    import numpy as np
+
+    def t(a, dt):
+        return torch.from_numpy(np.ascontiguousarray(a).view(dt))
+
+    out = [t(hidden_bits, np.int16).to(device).view(torch.bfloat16),
+           t(W_bits, np.int16).to(device).view(torch.bfloat16),
+           t(topk_idx, np.int32).to(device),
+           t(topk_logit, np.float32).to(device),
+           None if row_mask is None else t(row_mask, np.uint8).to(device)]
+    return tuple(out)

@@ -1,0 +1,155 @@
+/*
+ * fckl.h -- fused chunked forward-KL distillation loss on B200 (sm_100a).
+ *
+ * The operation (notation of the library):
+ *   rows r = 0..N-1 are the flattened batch x sequence positions; a row is valid
+ *   when row_mask[r] != 0 (all rows when row_mask is NULL); N_v = #valid rows.
+ *   z_r   = W h_r                         student logits over the vocabulary V
+ *   q     = softmax(z_r / T)              over all V
+ *   p     = softmax(topk_logit[r,:] / T)  over the K cached teacher ids, zero
+ *                                         elsewhere
+ *   l_r   = sum_k p_k (log p_k - log q[topk_idx[r,k]])     forward KL(p || q)
+ *   loss  = (1/N_v) sum_{valid r} l_r                      (0 when N_v = 0)
+ *   dH_r  = dlogits_r W,  dW = sum_r dlogits_r^T h_r,
+ *   dlogits_r = (q - p~) / (T N_v),  p~_v = sum_{k: topk_idx[r,k] = v} p_k,
+ *   and dlogits_r = 0 for masked rows.
+ *
+ * Passages this implements:
+ *   - "[논문리뷰] Efficient Knowledge Distillation for LLMs: Offline Top-K Logits
+ *     and a Fused Chunked KL Loss", section 1 (Key Terms): the output projection
+ *     is folded into the loss and the sequence is processed chunk by chunk, so
+ *     the full-vocabulary logit tensor is never created; section 3: memory is
+ *     linear in the sequence length.
+ *   - aibase.it write-up "Knowledge Distillation 비용 줄이기", section
+ *     "offline top-K logits 방식": the teacher is a per-position top-K cache of
+ *     token ids and logits (top-100); section "chunked KL loss가 하는 일": per
+ *     chunk, project hidden states to logits, add to the loss, discard, and
+ *     recompute the chunk in the backward pass.
+ *   - LLM Primer ch.6 "프루닝과 지식 증류", section 6.2: forward KL between the
+ *     temperature-softened teacher and student.
+ *   The pages give no formula for the gradient scale; this library applies no
+ *   T^2 factor (the gradients are those of `loss` itself, upstream grad 1).
+ *
+ * Common conventions for every entry point:
+ *   - All array pointers are DEVICE pointers into memory the caller owns; the
+ *     library allocates nothing (device or host) and keeps no state between
+ *     calls except a per-device cache of kernel attributes.
+ *   - Arrays are dense and row-major.  hidden, W, dH and dW must start on a
+ *     16-byte boundary (TMA), the others on a 4-byte boundary:
+ *       hidden     bf16  [N, H]      (raw bfloat16 bit patterns)
+ *       W          bf16  [V, H]
+ *       topk_idx   int32 [N, K]      ids in [0, V); order within a row is free
+ *       topk_logit fp32  [N, K]      may hold -inf (probability 0); not all -inf
+ *       row_mask   uint8 [N] or NULL
+ *       loss       fp32  scalar
+ *       row_loss   fp32  [N] or NULL (per-row l_r, 0 for masked rows)
+ *       dH         fp32  [N, H]      overwritten
+ *       dW         fp32  [V, H]      overwritten
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *     asynchronous on that stream; the workspace must not be shared by calls
+ *     that can overlap.
+ *   - Errors that the host can see (null pointers, bad sizes, misalignment,
+ *     T <= 0 or not finite, K > FCKL_K_MAX, H % 8 != 0, workspace too small)
+ *     are returned before anything is enqueued.  Errors only the device can see
+ *     (an id outside [0, V), a teacher row with no finite logit, an exhausted
+ *     bounded wait) are recorded in the workspace and reported by fckl_check().
+ */
+#ifndef FCKL_H_
+#define FCKL_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FCKL_K_MAX 256
+
+typedef enum {
+  FCKL_OK = 0,
+  FCKL_ERR_INVALID_ARG = 1,   /* null pointer, size <= 0, misaligned, T not > 0 */
+  FCKL_ERR_UNSUPPORTED = 2,   /* K > FCKL_K_MAX, H % 8 != 0, no sm_100 device   */
+  FCKL_ERR_WORKSPACE = 3,     /* workspace NULL or smaller than required        */
+  FCKL_ERR_BAD_INDEX = 4,     /* device: a topk_idx entry outside [0, V)        */
+  FCKL_ERR_BAD_TEACHER = 5,   /* device: a valid row whose K logits are NaN,
+                                 +inf, or all -inf                               */
+  FCKL_ERR_TIMEOUT = 6,       /* device: a bounded wait inside a kernel ran out */
+  FCKL_ERR_CUDA = 7           /* a CUDA runtime call or launch failed           */
+} fckl_status;
+
+/* Problem description.  chunk = rows per chunk (0 = automatic: the largest
+ * multiple of 128 rows whose bf16 dlogits block [chunk, V] fits in 512 MiB,
+ * capped at N rounded up to 64).  Live device bytes are O(chunk * V) for the
+ * workspace plus the caller's O(V * H) weights and gradients. */
+typedef struct {
+  int64_t N;      /* rows (batch * sequence)      */
+  int64_t H;      /* hidden size                  */
+  int64_t V;      /* vocabulary size              */
+  int32_t K;      /* cached teacher ids per row   */
+  float T;        /* temperature (> 0)            */
+  int64_t chunk;  /* rows per chunk, 0 = auto     */
+} fckl_problem;
+
+/* Bytes of device workspace fckl_fwd / fckl_fwd_bwd need for `prob` (0 when the
+ * problem is invalid).  Pure host arithmetic; needs no GPU. */
+size_t fckl_workspace_bytes(const fckl_problem* prob);
+
+/* The chunk size the library will use for `prob` (resolves chunk = 0), or -1
+ * when the problem is invalid.  Pure host arithmetic. */
+int64_t fckl_resolved_chunk(const fckl_problem* prob);
+
+/* Forward only: loss (and optionally row_loss).  Per chunk: teacher softmax
+ * over the K cached logits, the fused projection z = h W^T on the tensor cores
+ * with a full-vocabulary online log-sum-exp and a gather of z at the cached
+ * ids (the [chunk, V] logit tile is never written), then the per-row KL.
+ * Cost: 2*H*V flops per row. */
+fckl_status fckl_fwd(const fckl_problem* prob, const void* hidden, const void* W,
+                     const int32_t* topk_idx, const float* topk_logit,
+                     const uint8_t* row_mask, float* loss, float* row_loss,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* Forward + backward: loss, row_loss (optional), dH and dW (fp32, overwritten).
+ * Per chunk, after the forward steps above: recompute the logit tile, form
+ * bf16 dlogits = q - p~ (masked rows 0) in the GEMM epilogue, then
+ * dH_chunk = (1/(T N_v)) dlogits W and dW += (1/(T N_v)) dlogits^T h_chunk on
+ * the tensor cores with fp32 accumulation.  Cost: 8*H*V flops per row. */
+fckl_status fckl_fwd_bwd(const fckl_problem* prob, const void* hidden, const void* W,
+                         const int32_t* topk_idx, const float* topk_logit,
+                         const uint8_t* row_mask, float* loss, float* row_loss,
+                         float* dH, float* dW,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, then returns the first device-side error recorded in
+ * `workspace` by the last call that used it (FCKL_OK if none), or
+ * FCKL_ERR_CUDA if the stream reports a CUDA error. */
+fckl_status fckl_check(void* workspace, void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* fckl_status_string(fckl_status status);
+
+/* Optional per-kernel timing for measurement tools.  Between
+ * fckl_profile_begin() and fckl_profile_end(), every kernel the library
+ * launches is bracketed by two CUDA events recorded on the call's stream
+ * (events are created on first use and reused; no device memory is
+ * allocated).  fckl_profile_end() synchronises those events, stops recording
+ * and writes up to `max_stats` per-kernel summaries (one per kernel kind, in
+ * first-launch order); it returns how many kinds were seen, or -1 on a CUDA
+ * error.  Recording is process-wide and not thread-safe. */
+typedef struct {
+  char name[32];     /* kernel kind, e.g. "fwd_logits_lse" */
+  int64_t launches;  /* launches recorded */
+  double total_ms;   /* sum of event-timed durations */
+  double flops;      /* algorithmic flops of those launches (GEMMs: 2*M*N*K) */
+  double bytes;      /* algorithmic HBM bytes of those launches (compulsory
+                        reads + writes of operands and outputs) */
+} fckl_kernel_stat;
+
+void fckl_profile_begin(void);
+int fckl_profile_end(fckl_kernel_stat* stats, int max_stats);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FCKL_H_ */

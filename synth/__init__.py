@@ -18,7 +18,8 @@ Recipe (all streams are children of ``np.random.SeedSequence(1000 + cfg)``):
   stream 1  W        f32 normal(0, 0.02), [V, H], rounded to bf16 (RNE)
   stream 2  ids      per row K distinct ids, uniform in [0, V): a row of K
                      uniform integers is redrawn whole until it has no repeat
-                     (exact rejection sampling of an ordered distinct K-tuple)
+                     (exact rejection sampling of an ordered distinct K-tuple);
+                     when K^2 > 2V each row is drawn without replacement instead
   stream 3  logits   f32 normal(0, sigma), [N, K], each row sorted descending
                      and paired with the ids in draw order
   stream 4  mask     exactly round(f * N) rows set to 0, chosen without
@@ -106,6 +107,8 @@ def _normal_bf16(rng: np.random.Generator, rows: int, cols: int, scale: float) -
 
 
 def _distinct_ids(rng: np.random.Generator, rows: int, V: int, K: int) -> np.ndarray:
+    if K * K > 2 * V:  # repeats would be common: draw each row without replacement
+        return np.stack([rng.choice(V, size=K, replace=False) for _ in range(rows)]).astype(np.int32)
     ids = rng.integers(0, V, size=(rows, K), dtype=np.int64)
     while True:
         s = np.sort(ids, axis=1)

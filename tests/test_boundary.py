@@ -1,0 +1,125 @@
+"""C-ABI boundary checks that need no GPU: the library loads, exports every
+function the header declares, sizes its workspace, and rejects bad arguments
+before it touches the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import chunked_kl_loss_tcgen05_b200 as fk
+from chunked_kl_loss_tcgen05_b200 import FcklProblem
+from chunked_kl_loss_tcgen05_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fckl.h")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build()
+    return fk.load()
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(fckl_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_expected_api():
+    assert _declared_functions() == sorted(fk.exported_symbols)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(fk.lib_path())
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings():
+    for code in range(8):
+        s = fk.fckl_status_string(code)
+        assert s.startswith("FCKL_")
+    assert fk.fckl_status_string(0) == "FCKL_OK"
+    assert fk.fckl_status_string(99) == "FCKL_ERR_UNKNOWN"
+
+
+def test_workspace_and_chunk_rules():
+    p1 = FcklProblem(8192, 3072, 128256, 100, 1.0, 0)
+    assert fk.fckl_resolved_chunk(p1) == 2048          # 512 MiB of bf16 dlogits
+    p3 = FcklProblem(131072, 2880, 201088, 100, 1.0, 0)
+    assert fk.fckl_resolved_chunk(p3) == 1280
+    p0 = FcklProblem(256, 256, 4096, 16, 1.0, 64)
+    assert fk.fckl_resolved_chunk(p0) == 64
+    assert fk.fckl_resolved_chunk(FcklProblem(100, 256, 4096, 16, 1.0, 0)) == 100
+    assert fk.fckl_resolved_chunk(FcklProblem(100, 256, 4096, 16, 1.0, 4096)) == 100
+    # workspace holds the chunk's bf16 dlogits block and is linear in N beyond it
+    w = fk.fckl_workspace_bytes(p1)
+    assert w >= 2048 * 128256 * 2
+    a = fk.fckl_workspace_bytes(FcklProblem(32768, 4096, 128256, 100, 1.0, 1024))
+    b = fk.fckl_workspace_bytes(FcklProblem(65536, 4096, 128256, 100, 1.0, 1024))
+    assert b - a == 32768 * 4                           # only the per-row loss grows
+    assert a < 300 * 2**20
+
+
+@pytest.mark.parametrize("bad", [
+    dict(N=0), dict(H=0), dict(V=0), dict(K=0), dict(T=0.0), dict(T=-1.0),
+    dict(T=float("nan")), dict(T=float("inf")), dict(chunk=-1)])
+def test_invalid_problem_rejected(bad):
+    kw = dict(N=64, H=64, V=512, K=8, T=1.0, chunk=0)
+    kw.update(bad)
+    p = FcklProblem(**kw)
+    assert fk.fckl_workspace_bytes(p) == 0
+    assert fk.fckl_resolved_chunk(p) == -1
+    fake = 1 << 20
+    st = fk.fckl_fwd_bwd(p, fake, fake, fake, fake, None, fake, None, fake, fake, fake, 1 << 40, None)
+    assert st == fk.FCKL_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("bad", [dict(K=257), dict(H=60), dict(K=600, V=512)])
+def test_unsupported_problem_rejected(bad):
+    kw = dict(N=64, H=64, V=512, K=8, T=1.0, chunk=0)
+    kw.update(bad)
+    p = FcklProblem(**kw)
+    fake = 1 << 20
+    st = fk.fckl_fwd_bwd(p, fake, fake, fake, fake, None, fake, None, fake, fake, fake, 1 << 40, None)
+    assert st == fk.FCKL_ERR_UNSUPPORTED
+
+
+def test_null_and_misaligned_pointers_rejected():
+    p = FcklProblem(64, 64, 512, 8, 1.0, 0)
+    ws = fk.fckl_workspace_bytes(p)
+    f = 1 << 20
+    args = [f, f, f, f, None, f, None, f, f, f, ws]
+    for i in (0, 1, 2, 3, 5, 7, 8):
+        a = list(args)
+        a[i] = None
+        assert fk.fckl_fwd_bwd(p, *a, None) == fk.FCKL_ERR_INVALID_ARG, i
+    a = list(args)
+    a[0] = f + 8  # hidden must be 16-byte aligned for TMA
+    assert fk.fckl_fwd_bwd(p, *a, None) == fk.FCKL_ERR_INVALID_ARG
+    # forward-only does not need gradient buffers
+    st = fk.fckl_fwd(p, f, f, f, f, None, f, None, None, ws, None)
+    assert st == fk.FCKL_ERR_WORKSPACE
+
+
+def test_small_workspace_rejected():
+    p = FcklProblem(64, 64, 512, 8, 1.0, 0)
+    ws = fk.fckl_workspace_bytes(p)
+    f = 1 << 20
+    assert fk.fckl_fwd_bwd(p, f, f, f, f, None, f, None, f, f, f, ws - 1, None) == fk.FCKL_ERR_WORKSPACE
+    assert fk.fckl_fwd(p, f, f, f, f, None, f, None, f + 16, ws, None) == fk.FCKL_ERR_WORKSPACE
+
+
+def test_no_gpu_fails_loudly():
+    """With every argument valid and no usable sm_100 device the call refuses;
+    there is no host fallback."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    p = FcklProblem(64, 64, 512, 8, 1.0, 0)
+    ws = fk.fckl_workspace_bytes(p)
+    f = 1 << 20
+    st = fk.fckl_fwd_bwd(p, f, f, f, f, None, f, None, f, f, f, ws, None)
+    assert st in (fk.FCKL_ERR_UNSUPPORTED, fk.FCKL_ERR_CUDA)

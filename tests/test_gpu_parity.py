@@ -1,0 +1,197 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded inputs.
+
+Tolerances (stated for the method): loss within 1e-3 relative error; dH and dW
+within 2e-2 relative Frobenius error (bf16 inputs, fp32 accumulation).  The
+expected error is far smaller: logits are bf16 x bf16 products accumulated in
+fp32 (~1e-6 relative), and the gradients carry one bf16 rounding of dlogits
+(~2^-9 relative per element, averaging out in the products).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from chunked_kl_loss_tcgen05_b200 import FcklProblem, fckl_check, fckl_fwd_bwd, FCKL_OK
+from chunked_kl_loss_tcgen05_b200 import FCKL_ERR_BAD_INDEX, FCKL_ERR_BAD_TEACHER
+from chunked_kl_loss_tcgen05_b200.torch_api import (alloc_workspace, arrays_to_device,
+                                                    fused_kl_fwd, fused_kl_fwd_bwd)
+
+pytestmark = pytest.mark.gpu
+
+LOSS_RTOL = 1e-3
+GRAD_RTOL = 2e-2
+
+
+def rel_fro(a, b):
+    a = np.asarray(a, np.float64); b = np.asarray(b, np.float64)
+    nb = np.linalg.norm(b)
+    return np.linalg.norm(a - b) / nb if nb > 0 else np.linalg.norm(a)
+
+
+def run_gpu(inp, chunk=None, T=None, fwd_only=False, row_loss=True):
+    d = arrays_to_device(inp.hidden, inp.W, inp.topk_idx, inp.topk_logit, inp.row_mask)
+    T = inp.cfg.T if T is None else T
+    chunk = inp.cfg.chunk if chunk is None else chunk
+    if fwd_only:
+        loss, rl = fused_kl_fwd(*d, T=T, chunk=chunk, want_row_loss=row_loss)
+        torch.cuda.synchronize()
+        return dict(loss=loss.item(), row_loss=rl.cpu().numpy())
+    loss, rl, dH, dW = fused_kl_fwd_bwd(*d, T=T, chunk=chunk, want_row_loss=row_loss)
+    torch.cuda.synchronize()
+    return dict(loss=loss.item(), row_loss=rl.cpu().numpy(), dH=dH, dW=dW)
+
+
+def check_full(inp, g, o):
+    m = inp.row_mask != 0
+    assert abs(g["loss"] - o["loss"]) <= LOSS_RTOL * abs(o["loss"]), (g["loss"], o["loss"])
+    np.testing.assert_allclose(g["row_loss"][m], o["row_loss"][m], rtol=LOSS_RTOL, atol=1e-4)
+    assert (g["row_loss"][~m] == 0).all()
+    eh = rel_fro(g["dH"].cpu().numpy(), o["dH"])
+    ew = rel_fro(g["dW"].cpu().numpy(), o["dW"])
+    assert eh <= GRAD_RTOL and ew <= GRAD_RTOL, (eh, ew)
+    return eh, ew
+
+
+def test_tiny_config_full():
+    inp = synth.make_inputs(0)
+    o = oracle.oracle_from_inputs(inp)
+    g = run_gpu(inp)
+    eh, ew = check_full(inp, g, o)
+    assert eh < 5e-3 and ew < 5e-3, (eh, ew)   # far inside the stated bound
+
+
+@pytest.mark.parametrize("chunk", [64, 100, 128, 256, 0])
+def test_tiny_config_chunk_invariance(chunk):
+    """Chunking rows differently gives the same loss and gradients."""
+    inp = synth.make_inputs(0)
+    ref = run_gpu(inp, chunk=256)
+    g = run_gpu(inp, chunk=chunk)
+    assert abs(g["loss"] - ref["loss"]) <= 1e-5 * abs(ref["loss"])
+    np.testing.assert_allclose(g["row_loss"], ref["row_loss"], rtol=1e-5, atol=1e-6)
+    assert rel_fro(g["dH"].cpu().numpy(), ref["dH"].cpu().numpy()) < 1e-5
+    assert rel_fro(g["dW"].cpu().numpy(), ref["dW"].cpu().numpy()) < 1e-5
+
+
+EDGE = [
+    # name, N, H, V, K, T, mask_frac, chunk
+    ("ragged_rows", 333, 128, 2048, 16, 1.0, 0.1, 128),
+    ("vocab_tail", 200, 128, 1000, 8, 1.0, 0.0, 0),
+    ("vocab_not_mult8", 130, 64, 1003, 5, 0.7, 0.0, 64),
+    ("hidden_tail", 150, 200, 777, 12, 1.3, 0.2, 96),
+    ("hidden_small", 64, 8, 300, 4, 1.0, 0.0, 0),
+    ("k_one", 256, 256, 4096, 1, 1.0, 0.0, 0),
+    ("k_max", 129, 64, 600, 256, 2.0, 0.0, 0),
+    ("temperature_2", 256, 256, 4096, 16, 2.0, 0.25, 64),
+    ("one_row", 1, 64, 512, 3, 1.0, 0.0, 0),
+    ("many_chunks", 1000, 64, 513, 7, 1.0, 0.05, 37),
+]
+
+
+@pytest.mark.parametrize("case", EDGE, ids=[c[0] for c in EDGE])
+def test_edge_shapes(case):
+    name, N, H, V, K, T, mf, chunk = case
+    seed = 100 + [c[0] for c in EDGE].index(name)
+    inp = synth.make_custom(N, H, V, K, T=T, sigma=2.0, mask_frac=mf, seed=seed, chunk=chunk)
+    o = oracle.oracle_from_inputs(inp)
+    g = run_gpu(inp)
+    check_full(inp, g, o)
+
+
+def test_forward_only_matches():
+    inp = synth.make_inputs(0)
+    a = run_gpu(inp, fwd_only=True)
+    b = run_gpu(inp)
+    assert a["loss"] == pytest.approx(b["loss"], rel=1e-6)
+    np.testing.assert_allclose(a["row_loss"], b["row_loss"], rtol=1e-6, atol=1e-7)
+
+
+def test_no_valid_rows():
+    inp = synth.make_custom(100, 64, 512, 8, mask_frac=1.0, seed=3)
+    g = run_gpu(inp)
+    assert g["loss"] == 0.0
+    assert not g["dH"].any().item() and not g["dW"].any().item()
+
+
+def test_masked_rows_do_not_matter():
+    inp = synth.make_custom(300, 128, 2000, 10, mask_frac=0.3, seed=4, chunk=128)
+    g1 = run_gpu(inp)
+    m = inp.row_mask == 0
+    rng = np.random.default_rng(0)
+    inp.hidden[m] = synth.f32_to_bf16_bits(rng.standard_normal((m.sum(), 128)).astype(np.float32) * 5)
+    inp.topk_logit[m] = rng.standard_normal((m.sum(), 10)).astype(np.float32) * 7
+    g2 = run_gpu(inp)
+    assert g1["loss"] == g2["loss"]
+    assert rel_fro(g2["dW"].cpu().numpy(), g1["dW"].cpu().numpy()) < 1e-6
+    assert g2["dH"][torch.from_numpy(m).cuda()].abs().max().item() == 0.0
+
+
+def test_llama_8k_config_full():
+    inp = synth.make_inputs(1)
+    g = run_gpu(inp)
+    o = oracle.oracle_from_inputs(inp)
+    check_full(inp, g, o)
+
+
+@pytest.mark.parametrize("cfg", [2, 3, 4])
+def test_large_config_sampled_rows(cfg):
+    """Full-size configs: per-row loss and dH on 64 seeded valid rows against
+    the oracle; the mean of the row losses, the zero column sums of dW and the
+    zero dH of masked rows at full size."""
+    inp = synth.make_inputs(cfg)
+    rows = synth.sample_rows(inp, 64)
+    g = run_gpu(inp)
+    o = oracle.oracle_from_inputs(inp, rows=rows)
+    np.testing.assert_array_equal(o["rows"], rows)
+    np.testing.assert_allclose(g["row_loss"][rows], o["row_loss_rows"], rtol=LOSS_RTOL, atol=1e-4)
+    dH_rows = g["dH"][torch.from_numpy(rows).cuda()].cpu().numpy()
+    assert rel_fro(dH_rows, o["dH_rows"]) <= GRAD_RTOL
+    m = inp.row_mask != 0
+    mean = g["row_loss"][m].astype(np.float64).mean()
+    assert abs(g["loss"] - mean) <= 1e-5 * abs(mean)
+    if (~m).any():
+        assert g["dH"][torch.from_numpy(~m).cuda()].abs().max().item() == 0.0
+    dW = g["dW"]
+    colsum = dW.double().sum(dim=0)
+    scale = dW.double().abs().sum(dim=0)
+    assert (colsum.abs() <= 2e-2 * scale + 1e-30).all().item()
+    del g, dW
+    torch.cuda.empty_cache()
+
+
+def _raw_call(inp, ids=None, logits=None):
+    d = list(arrays_to_device(inp.hidden, inp.W, inp.topk_idx if ids is None else ids,
+                              inp.topk_logit if logits is None else logits, inp.row_mask))
+    p = FcklProblem(inp.cfg.N, inp.cfg.H, inp.cfg.V, inp.cfg.K, inp.cfg.T, inp.cfg.chunk)
+    ws = alloc_workspace(p, "cuda")
+    loss = torch.empty(1, device="cuda")
+    dH = torch.empty(inp.cfg.N, inp.cfg.H, device="cuda")
+    dW = torch.empty(inp.cfg.V, inp.cfg.H, device="cuda")
+    st = fckl_fwd_bwd(p, d[0].data_ptr(), d[1].data_ptr(), d[2].data_ptr(), d[3].data_ptr(),
+                      None if d[4] is None else d[4].data_ptr(), loss.data_ptr(), None,
+                      dH.data_ptr(), dW.data_ptr(), ws.data_ptr(), ws.numel(),
+                      torch.cuda.current_stream().cuda_stream)
+    assert st == FCKL_OK
+    return fckl_check(ws.data_ptr(), torch.cuda.current_stream().cuda_stream)
+
+
+def test_out_of_range_id_is_reported():
+    inp = synth.make_custom(64, 64, 512, 8, seed=5)
+    assert _raw_call(inp) == FCKL_OK
+    ids = inp.topk_idx.copy()
+    ids[17, 3] = 512
+    assert _raw_call(inp, ids=ids) == FCKL_ERR_BAD_INDEX
+    ids = inp.topk_idx.copy()
+    ids[5, 0] = -1
+    assert _raw_call(inp, ids=ids) == FCKL_ERR_BAD_INDEX
+
+
+def test_teacher_row_without_finite_logit_is_reported():
+    inp = synth.make_custom(64, 64, 512, 8, seed=6)
+    lg = inp.topk_logit.copy()
+    lg[9, :] = -np.inf
+    assert _raw_call(inp, logits=lg) == FCKL_ERR_BAD_TEACHER
+    lg = inp.topk_logit.copy()
+    lg[3, 2] = np.nan
+    assert _raw_call(inp, logits=lg) == FCKL_ERR_BAD_TEACHER
