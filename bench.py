@@ -49,7 +49,7 @@ def load_peaks():
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--config", type=int, default=1)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
@@ -207,14 +207,13 @@ def run_cuda(args):
     def step():
         return fused_kl_fwd_bwd(*d, T=cfg.T, chunk=cfg.chunk, workspace=ws, check=False)
 
-    for _ in range(args.warmup):
-        out = step()
-    torch.cuda.synchronize()
     from chunked_kl_loss_tcgen05_b200 import fckl_check
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
     st = fckl_check(ws.data_ptr(), torch.cuda.current_stream().cuda_stream)
     if st != 0:
         raise SystemExit(f"device error after warm-up: status {st}")
-    del out
 
     clocks = ClockSampler(local)
     stream = torch.cuda.current_stream(dev)
@@ -235,6 +234,9 @@ def run_cuda(args):
     peak_gib = torch.cuda.max_memory_allocated(dev) / 2**30
     loss_val = float(out[0].item())
     del out
+    st = fckl_check(ws.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    if st != 0:
+        raise SystemExit(f"device error in the timed steps: status {st}")
 
     t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
     if world > 1:

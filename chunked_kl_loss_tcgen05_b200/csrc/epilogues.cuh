@@ -7,11 +7,20 @@
 //               z at the row's cached teacher ids.  Nothing of the tile is
 //               written; one (max, sum) partial per row per vocab segment.
 //   EpiDlogits  backward: recomputed z tile -> q - p~ (0 for masked rows and
-//               for columns >= V), rounded once to bf16, stored to the chunk's
-//               dlogits block.
-//   EpiDH       dH[rows, :] += alpha * (dlogits W) partial (split-K), fp32.
-//   EpiDW       dW (+)= alpha * (dlogits^T h), fp32 read-modify-write.
+//               for columns >= V), rounded once to bf16, staged in shared
+//               memory and TMA-stored to the chunk's dlogits block.
+//   EpiDH       dH[rows, :] += alpha * (dlogits W) partial (split-K): fp32
+//               tile staged in shared memory, TMA reduce-add into dH.
+//   EpiDW       dW (+)= alpha * (dlogits^T h): TMA store (first chunk) or
+//               TMA reduce-add (later chunks), so the fp32 read-modify-write
+//               of dW happens in L2, coalesced and off the epilogue threads.
 // alpha = 1 / (T * N_valid) is applied here so the bf16 operand stays O(1).
+//
+// Staging layout (EpiDlogits / EpiDH / EpiDW): each epilogue warp owns two
+// 4 KB buffers (double buffering against the TMA engine).  A buffer holds the
+// warp's 32 rows x 128 bytes in the TMA 128-byte swizzle: the 16-byte chunk j
+// of row r sits at r * 128 + ((j ^ (r & 7)) * 16), which also makes the
+// per-thread row writes bank-conflict free.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -37,6 +46,8 @@ __device__ __forceinline__ void tmem_ld32_conv(uint32_t taddr, float (&v)[32]) {
 }
 
 struct EpiLse {
+  static constexpr uint32_t kSmemBytes = 0;
+  static constexpr bool kUsesMapC = false;
   struct Params {
     int rows_c;      // valid rows of this chunk
     int V, K, Smax;
@@ -49,10 +60,11 @@ struct EpiLse {
     float m, s;
     int cur, nid;
   };
-  static __device__ void init(const Params&, State& st) {
+  static __device__ void init(const Params&, State& st, uint8_t*, int) {
     st.m = -INFINITY; st.s = 0.f; st.cur = 0; st.nid = INT_MAX;
   }
-  static __device__ void tile(const Params& p, State& st, const Work& w, uint32_t taddr, int r) {
+  static __device__ void tile(const Params& p, State& st, const Work& w, uint32_t taddr, int r,
+                              const CUtensorMap*, int, int) {
     const int row = w.mb * BM + r;
     const bool rv = row < p.rows_c;
     const int* rid = p.sid + (size_t)(rv ? row : 0) * p.K;
@@ -102,7 +114,7 @@ struct EpiLse {
     if (w.seg_end && rv)
       p.partials[((size_t)w.mb * p.Smax + w.split) * BM + r] = make_float2(st.m, st.s);
   }
-  static __device__ void finish(const Params&, State&) {}
+  static __device__ void finish(const Params&, State&, int) {}
 };
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -110,21 +122,68 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&b);
 }
 
+// Swizzled position of 16-byte chunk j of this lane's row in a staging buffer.
+__device__ __forceinline__ uint4* stage_chunk(uint8_t* buf, int lane, int j) {
+  return reinterpret_cast<uint4*>(buf + lane * 128 + ((j ^ (lane & 7)) << 4));
+}
+
+// Wait until the staging buffer about to be refilled is no longer read by the
+// TMA store issued two slices ago (only the issuing lane can wait on it).
+__device__ __forceinline__ void stage_acquire(int lane) {
+  if (lane == 0) bulk_wait_read<1>();
+  __syncwarp();
+}
+// Publish this warp's staged rows to the TMA engine.
+__device__ __forceinline__ void stage_release() {
+  fence_async_smem();
+  __syncwarp();
+}
+
 struct EpiDlogits {
+  static constexpr uint32_t kSmemBytes = 4 * 2 * 4096;
+  static constexpr bool kUsesMapC = true;  // map C: dlogits [rows_c, V] bf16, box {64, 32}
   struct Params {
-    int rows_c, V, Vp, K;
+    int rows_c, V, K;
     float scale2;          // log2(e) / T
     const float* lse2;     // [rows_c] log2-domain log-sum-exp of z / T
     const int* sid;        // [rows_c, K] sorted ids
     const float* sp;       // [rows_c, K] teacher probabilities, same order
     const uint8_t* mask;   // chunk rows, or nullptr
-    __nv_bfloat16* dlog;   // [rows_c, Vp]
   };
   struct State {
-    int cur, nid;
+    int cur, nid, n;
+    uint8_t* buf;
   };
-  static __device__ void init(const Params&, State& st) { st.cur = 0; st.nid = INT_MAX; }
-  static __device__ void tile(const Params& p, State& st, const Work& w, uint32_t taddr, int r) {
+  static __device__ void init(const Params&, State& st, uint8_t* smem_warp, int) {
+    st.cur = 0; st.nid = INT_MAX; st.n = 0; st.buf = smem_warp;
+  }
+  // q - p~ for one 32-column slice in place (v holds raw z on entry).
+  static __device__ __forceinline__ void slice(const Params& p, State& st, float (&v)[32],
+                                               int base, bool keep, float lse, const int* rid,
+                                               const float* rp) {
+    if (!keep) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = 0.f;
+      return;
+    }
+    if (base + 32 <= p.V) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = exp2f(fmaf(v[j], p.scale2, -lse));
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = (base + j < p.V) ? exp2f(fmaf(v[j], p.scale2, -lse)) : 0.f;
+    }
+    while (st.nid < base + 32) {  // subtract the teacher mass at cached ids
+      const int j = st.nid - base;
+      const float pv = __ldg(rp + st.cur);
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) v[jj] = (jj == j) ? v[jj] - pv : v[jj];
+      ++st.cur;
+      st.nid = st.cur < p.K ? __ldg(rid + st.cur) : INT_MAX;
+    }
+  }
+  static __device__ void tile(const Params& p, State& st, const Work& w, uint32_t taddr, int r,
+                              const CUtensorMap* mapC, int quarter, int lane) {
     const int row = w.mb * BM + r;
     const bool rv = row < p.rows_c;
     const bool keep = rv && (p.mask == nullptr || p.mask[row] != 0);
@@ -132,128 +191,140 @@ struct EpiDlogits {
     const float* rp = p.sp + (size_t)(rv ? row : 0) * p.K;
     const float lse = keep ? p.lse2[row] : 0.f;
     const int col0 = w.nb * BN;
+    const int y = w.mb * BM + quarter * 32;
     if (w.seg_begin && keep) {
       st.cur = lower_bound_ids(rid, p.K, col0);
       st.nid = st.cur < p.K ? __ldg(rid + st.cur) : INT_MAX;
     }
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
-      float v[32];
-      tmem_ld32_conv(taddr + (uint32_t)(c * 32), v);
-      const int base = col0 + c * 32;
-      if (!rv || base >= p.Vp) continue;
-      if (keep) {
-        if (base + 32 <= p.V) {
+    for (int s = 0; s < BN / 64; ++s) {
+      const int base = col0 + s * 64;
+      float v0[32], v1[32];
+      tmem_ld32_conv(taddr + (uint32_t)(s * 64), v0);
+      tmem_ld32_conv(taddr + (uint32_t)(s * 64 + 32), v1);
+      slice(p, st, v0, base, keep, lse, rid, rp);
+      slice(p, st, v1, base + 32, keep, lse, rid, rp);
+      uint8_t* buf = st.buf + (st.n & 1) * 4096;
+      stage_acquire(lane);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = exp2f(fmaf(v[j], p.scale2, -lse));
-        } else {
+      for (int j = 0; j < 4; ++j)
+        *stage_chunk(buf, lane, j) = make_uint4(pack_bf16x2(v0[8 * j], v0[8 * j + 1]),
+                                                pack_bf16x2(v0[8 * j + 2], v0[8 * j + 3]),
+                                                pack_bf16x2(v0[8 * j + 4], v0[8 * j + 5]),
+                                                pack_bf16x2(v0[8 * j + 6], v0[8 * j + 7]));
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = (base + j < p.V) ? exp2f(fmaf(v[j], p.scale2, -lse)) : 0.f;
-        }
-        while (st.nid < base + 32) {  // subtract the teacher mass at cached ids
-          const int j = st.nid - base;
-          const float pv = __ldg(rp + st.cur);
-#pragma unroll
-          for (int jj = 0; jj < 32; ++jj) v[jj] = (jj == j) ? v[jj] - pv : v[jj];
-          ++st.cur;
-          st.nid = st.cur < p.K ? __ldg(rid + st.cur) : INT_MAX;
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = 0.f;
+      for (int j = 0; j < 4; ++j)
+        *stage_chunk(buf, lane, 4 + j) = make_uint4(pack_bf16x2(v1[8 * j], v1[8 * j + 1]),
+                                                    pack_bf16x2(v1[8 * j + 2], v1[8 * j + 3]),
+                                                    pack_bf16x2(v1[8 * j + 4], v1[8 * j + 5]),
+                                                    pack_bf16x2(v1[8 * j + 6], v1[8 * j + 7]));
+      stage_release();
+      if (lane == 0) {  // one group per slice, empty when the slice lies outside the map
+        if (base < p.V && y < p.rows_c) tma_store_2d(mapC, smem_u32(buf), base, y);
+        bulk_commit();
       }
-      uint4* dst = reinterpret_cast<uint4*>(p.dlog + (size_t)row * p.Vp + base);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        if (base + 8 * i < p.Vp) {
-          uint4 o;
-          o.x = pack_bf16x2(v[8 * i + 0], v[8 * i + 1]);
-          o.y = pack_bf16x2(v[8 * i + 2], v[8 * i + 3]);
-          o.z = pack_bf16x2(v[8 * i + 4], v[8 * i + 5]);
-          o.w = pack_bf16x2(v[8 * i + 6], v[8 * i + 7]);
-          dst[i] = o;
-        }
-      }
+      ++st.n;
     }
   }
-  static __device__ void finish(const Params&, State&) {}
+  static __device__ void finish(const Params&, State&, int lane) {
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
+  }
 };
 
+// Shared staging of alpha * accumulator, one 32-column fp32 slice at a time,
+// written to global memory by TMA (store or reduce-add).
+template <bool kReduce>
+__device__ __forceinline__ void stage_fp32_slices(uint8_t* bufs, int& n, uint32_t taddr,
+                                                  float alpha, const CUtensorMap* map, int x0,
+                                                  int x_end, int y, bool y_ok, int lane) {
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    float v[32];
+    tmem_ld32_conv(taddr + (uint32_t)(c * 32), v);
+    uint8_t* buf = bufs + (n & 1) * 4096;
+    stage_acquire(lane);
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      *stage_chunk(buf, lane, j) =
+          make_uint4(__float_as_uint(alpha * v[4 * j]), __float_as_uint(alpha * v[4 * j + 1]),
+                     __float_as_uint(alpha * v[4 * j + 2]), __float_as_uint(alpha * v[4 * j + 3]));
+    stage_release();
+    const int x = x0 + c * 32;
+    if (lane == 0) {  // one group per slice, empty when the slice lies outside the map
+      if (x < x_end && y_ok) {
+        if (kReduce) tma_reduce_add_2d(map, smem_u32(buf), x, y);
+        else tma_store_2d(map, smem_u32(buf), x, y);
+      }
+      bulk_commit();
+    }
+    ++n;
+  }
+}
+
 struct EpiDH {
+  static constexpr uint32_t kSmemBytes = 4 * 2 * 4096;
+  static constexpr bool kUsesMapC = true;  // map C: dH chunk rows [rows_c, H] fp32, box {32, 32}
   struct Params {
     int rows_c, H;
     float invT;
     const DeviceCtl* ctl;
-    float* dH;  // chunk rows: [rows_c, H]
   };
   struct State {
     float alpha;
+    int n;
+    uint8_t* buf;
   };
-  static __device__ void init(const Params& p, State& st) {
-    const int n = p.ctl->n_valid;
-    st.alpha = n > 0 ? p.invT / (float)n : 0.f;
+  static __device__ void init(const Params& p, State& st, uint8_t* smem_warp, int) {
+    const int nv = p.ctl->n_valid;
+    st.alpha = nv > 0 ? p.invT / (float)nv : 0.f;
+    st.n = 0;
+    st.buf = smem_warp;
   }
-  static __device__ void tile(const Params& p, State& st, const Work& w, uint32_t taddr, int r) {
-    const int row = w.mb * BM + r;
-    const bool rv = row < p.rows_c;
-#pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
-      float v[32];
-      tmem_ld32_conv(taddr + (uint32_t)(c * 32), v);
-      if (!rv) continue;
-      const int col = w.nb * BN + c * 32;
-      float* dst = p.dH + (size_t)row * p.H + col;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        if (col + 4 * i < p.H)
-          atomicAdd(reinterpret_cast<float4*>(dst + 4 * i),
-                    make_float4(st.alpha * v[4 * i], st.alpha * v[4 * i + 1],
-                                st.alpha * v[4 * i + 2], st.alpha * v[4 * i + 3]));
-      }
-    }
+  static __device__ void tile(const Params& p, State& st, const Work& w, uint32_t taddr, int,
+                              const CUtensorMap* mapC, int quarter, int lane) {
+    const int y = w.mb * BM + quarter * 32;
+    stage_fp32_slices<true>(st.buf, st.n, taddr, st.alpha, mapC, w.nb * BN, p.H, y,
+                            y < p.rows_c, lane);
   }
-  static __device__ void finish(const Params&, State&) {}
+  static __device__ void finish(const Params&, State&, int lane) {
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
+  }
 };
 
 struct EpiDW {
+  static constexpr uint32_t kSmemBytes = 4 * 2 * 4096;
+  static constexpr bool kUsesMapC = true;  // map C: dW [V, H] fp32, box {32, 32}
   struct Params {
     int V, H;
     float invT;
     int accumulate;  // 0: overwrite (first chunk), 1: add
     const DeviceCtl* ctl;
-    float* dW;       // [V, H]
   };
   struct State {
     float alpha;
+    int n;
+    uint8_t* buf;
   };
-  static __device__ void init(const Params& p, State& st) {
-    const int n = p.ctl->n_valid;
-    st.alpha = n > 0 ? p.invT / (float)n : 0.f;
+  static __device__ void init(const Params& p, State& st, uint8_t* smem_warp, int) {
+    const int nv = p.ctl->n_valid;
+    st.alpha = nv > 0 ? p.invT / (float)nv : 0.f;
+    st.n = 0;
+    st.buf = smem_warp;
   }
-  static __device__ void tile(const Params& p, State& st, const Work& w, uint32_t taddr, int r) {
-    const int vr = w.mb * BM + r;
-    const bool rv = vr < p.V;
-#pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
-      float v[32];
-      tmem_ld32_conv(taddr + (uint32_t)(c * 32), v);
-      if (!rv) continue;
-      const int col = w.nb * BN + c * 32;
-      float4* dst = reinterpret_cast<float4*>(p.dW + (size_t)vr * p.H + col);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        if (col + 4 * i < p.H) {
-          float4 o = p.accumulate ? dst[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-          o.x = fmaf(st.alpha, v[4 * i + 0], o.x);
-          o.y = fmaf(st.alpha, v[4 * i + 1], o.y);
-          o.z = fmaf(st.alpha, v[4 * i + 2], o.z);
-          o.w = fmaf(st.alpha, v[4 * i + 3], o.w);
-          dst[i] = o;
-        }
-      }
-    }
+  static __device__ void tile(const Params& p, State& st, const Work& w, uint32_t taddr, int,
+                              const CUtensorMap* mapC, int quarter, int lane) {
+    const int y = w.mb * BM + quarter * 32;
+    if (p.accumulate)
+      stage_fp32_slices<true>(st.buf, st.n, taddr, st.alpha, mapC, w.nb * BN, p.H, y, y < p.V, lane);
+    else
+      stage_fp32_slices<false>(st.buf, st.n, taddr, st.alpha, mapC, w.nb * BN, p.H, y, y < p.V, lane);
   }
-  static __device__ void finish(const Params&, State&) {}
+  static __device__ void finish(const Params&, State&, int lane) {
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
+  }
 };
 
 }  // namespace fckl

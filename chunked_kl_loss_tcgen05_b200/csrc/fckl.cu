@@ -100,19 +100,21 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// bf16 2-D map: inner (contiguous) extent, outer extent, outer stride in bytes,
-// box {box_inner, box_outer}, 128-byte swizzle, zero fill out of bounds.
+// 2-D map (bf16 or fp32): inner (contiguous) extent, outer extent, outer
+// stride in bytes, box {box_inner, box_outer}, 128-byte swizzle, zero fill out
+// of bounds.
 bool make_map(CUtensorMap* m, const void* base, long long inner, long long outer,
-              long long stride_bytes, int box_inner, int box_outer) {
+              long long stride_bytes, int box_inner, int box_outer, bool fp32 = false) {
   EncodeTiledFn enc = get_encode_fn();
   if (enc == nullptr) return false;
   cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
   cuuint64_t strides[1] = {(cuuint64_t)stride_bytes};
   cuuint32_t box[2] = {(cuuint32_t)box_inner, (cuuint32_t)box_outer};
   cuuint32_t estr[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return enc(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+             const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // ---------------------------------------------------------------- device info
@@ -128,7 +130,7 @@ template <class Sched, class Epi, bool A_MN, bool B_MN>
 bool set_smem_attr() {
   return cudaFuncSetAttribute(gemm_kernel<Sched, Epi, A_MN, B_MN>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)GEMM_SMEM_BYTES) == cudaSuccess;
+                              (int)gemm_smem_bytes<Epi>()) == cudaSuccess;
 }
 
 const DeviceInfo* device_info() {
@@ -277,9 +279,10 @@ fckl_status run(bool bwd, const fckl_problem* prob, const void* hidden, const vo
     k_count_valid<<<1, 1024, 0, st>>>(row_mask, L.N, ctl);
   }
 
-  CUtensorMap mapW_k, mapW_mn;
+  CUtensorMap mapW_k, mapW_mn, mapdW;
   if (!make_map(&mapW_k, W, L.H, L.V, L.H * 2, BK, BN)) return FCKL_ERR_CUDA;
   if (bwd && !make_map(&mapW_mn, W, L.H, L.V, L.H * 2, 64, BK)) return FCKL_ERR_CUDA;
+  if (bwd && !make_map(&mapdW, dW, L.H, L.V, L.H * 4, 32, 32, true)) return FCKL_ERR_CUDA;
 
   const long long NT = cdiv(L.V, BN);
   const long long KBh = cdiv(L.H, BK);
@@ -314,7 +317,8 @@ fckl_status run(bool bwd, const fckl_problem* prob, const void* hidden, const vo
     {
       ProfScope ps(K_FWD, st, gemm_flops, 2.0 * (rows + (double)L.V) * L.H + rows * K * 4.0);
       gemm_kernel<SchedLinear, EpiLse, false, false>
-          <<<G, GEMM_THREADS, GEMM_SMEM_BYTES, st>>>(mapH_k, mapW_k, pf, sa_lin, ca_f);
+          <<<G, GEMM_THREADS, gemm_smem_bytes<EpiLse>(), st>>>(mapH_k, mapW_k, mapW_k, pf,
+                                                               sa_lin, ca_f);
     }
 
     {
@@ -325,11 +329,14 @@ fckl_status run(bool bwd, const fckl_problem* prob, const void* hidden, const vo
     }
     if (!bwd) continue;
 
-    EpiDlogits::Params pb{rows, V, (int)L.Vp, K, scale2, lse2, sid, sp, mask_c, dlog};
+    EpiDlogits::Params pb{rows, V, K, scale2, lse2, sid, sp, mask_c};
+    CUtensorMap mapD_st;
+    if (!make_map(&mapD_st, dlog, L.V, rows, L.Vp * 2, 64, 32)) return FCKL_ERR_CUDA;
     {
-      ProfScope ps(K_BWD, st, gemm_flops, 2.0 * (rows + (double)L.V) * L.H + 2.0 * rows * L.Vp);
+      ProfScope ps(K_BWD, st, gemm_flops, 2.0 * (rows + (double)L.V) * L.H + 2.0 * rows * L.V);
       gemm_kernel<SchedLinear, EpiDlogits, false, false>
-          <<<G, GEMM_THREADS, GEMM_SMEM_BYTES, st>>>(mapH_k, mapW_k, pb, sa_lin, ca);
+          <<<G, GEMM_THREADS, gemm_smem_bytes<EpiDlogits>(), st>>>(mapH_k, mapW_k, mapD_st, pb,
+                                                                   sa_lin, ca);
     }
 
     // dH[rows] = alpha * dlogits W : A = dlogits (K-major), B = W (MN-major).
@@ -343,12 +350,15 @@ fckl_status run(bool bwd, const fckl_problem* prob, const void* hidden, const vo
     const int S = choose_split(tiles_h, KBv, dev->sms);
     SchedArgs sa_dh{tiles_h * S, (int)NTh, (int)KBv, S, (int)tiles_h};
     const int Gh = (int)std::min<long long>(dev->sms, tiles_h * S);
-    EpiDH::Params ph{rows, H, invT, ctl, dH + row0 * L.H};
+    EpiDH::Params ph{rows, H, invT, ctl};
+    CUtensorMap mapdH;
+    if (!make_map(&mapdH, dH + row0 * L.H, L.H, rows, L.H * 4, 32, 32, true)) return FCKL_ERR_CUDA;
     {
       ProfScope ps(K_DH, st, gemm_flops,
                    2.0 * rows * (double)L.V + 2.0 * (double)L.V * L.H + 4.0 * rows * L.H);
       gemm_kernel<SchedSplitK, EpiDH, false, true>
-          <<<Gh, GEMM_THREADS, GEMM_SMEM_BYTES, st>>>(mapD_k, mapW_mn, ph, sa_dh, ca);
+          <<<Gh, GEMM_THREADS, gemm_smem_bytes<EpiDH>(), st>>>(mapD_k, mapW_mn, mapdH, ph, sa_dh,
+                                                               ca);
     }
 
     // dW (+)= alpha * dlogits^T h : A = dlogits^T (MN-major), B = h (MN-major).
@@ -357,13 +367,14 @@ fckl_status run(bool bwd, const fckl_problem* prob, const void* hidden, const vo
     const long long tiles_w = cdiv(L.V, BM) * NTh;
     SchedArgs sa_dw{tiles_w, (int)NTh, (int)cdiv(rows, BK), 1, (int)tiles_w};
     const int Gw = (int)std::min<long long>(dev->sms, tiles_w);
-    EpiDW::Params pw{V, H, invT, c > 0 ? 1 : 0, ctl, dW};
+    EpiDW::Params pw{V, H, invT, c > 0 ? 1 : 0, ctl};
     {
       ProfScope ps(K_DW, st, gemm_flops,
                    2.0 * rows * (double)L.V + 2.0 * rows * L.H +
                        (c > 0 ? 8.0 : 4.0) * (double)L.V * L.H);
       gemm_kernel<SchedTiles, EpiDW, true, true>
-          <<<Gw, GEMM_THREADS, GEMM_SMEM_BYTES, st>>>(mapD_mn, mapH_mn, pw, sa_dw, ca);
+          <<<Gw, GEMM_THREADS, gemm_smem_bytes<EpiDW>(), st>>>(mapD_mn, mapH_mn, mapdW, pw, sa_dw,
+                                                               ca);
     }
   }
   {

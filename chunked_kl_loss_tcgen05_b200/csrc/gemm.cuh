@@ -31,7 +31,13 @@ constexpr uint32_t B_STAGE_BYTES = BN * BK * 2;  // 32 KB
 constexpr uint32_t STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int GEMM_THREADS = 192;
-constexpr size_t GEMM_SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+// Dynamic shared memory: 1 KB alignment slack, the operand stages, the
+// epilogue's staging area (Epi::kSmemBytes, split evenly over the 4 epilogue
+// warps) and 256 bytes of barriers.
+template <class Epi>
+constexpr size_t gemm_smem_bytes() {
+  return 1024 + (size_t)STAGES * STAGE_BYTES + Epi::kSmemBytes + 256;
+}
 
 // Wait-site codes recorded on timeout (diagnostics only).
 enum : uint32_t {
@@ -137,13 +143,15 @@ struct CtlArgs {
 template <class Sched, class Epi, bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const typename Epi::Params ep, const SchedArgs sa, const CtlArgs ca) {
+                const __grid_constant__ CUtensorMap tmC, const typename Epi::Params ep,
+                const SchedArgs sa, const CtlArgs ca) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_STAGE_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint8_t* sEpi = smem + STAGES * STAGE_BYTES;  // 1 KB aligned
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + Epi::kSmemBytes);
   uint64_t* full = bars;                // [STAGES]  TMA -> MMA
   uint64_t* empty = bars + STAGES;      // [STAGES]  MMA -> TMA
   uint64_t* tfull = bars + 2 * STAGES;  // [2]       MMA -> epilogue
@@ -169,6 +177,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (Epi::kUsesMapC) tma_prefetch_desc(&tmC);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
@@ -284,7 +293,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     typename Epi::State st;
-    Epi::init(ep, st);
+    Epi::init(ep, st, sEpi + quarter * (Epi::kSmemBytes / 4), lane);
     while (sch.next(w)) {
       bool ok = true;
       if (lane == 0) ok = wait_phase(smem_u32(&tfull[acc]), acc_phase, wc, SITE_EPI_TFULL);
@@ -292,14 +301,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       if (!ok) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
-      Epi::tile(ep, st, w, taddr, r);
+      Epi::tile(ep, st, w, taddr, r, &tmC, quarter, lane);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
-    Epi::finish(ep, st);
+    Epi::finish(ep, st, lane);
   }
 
   tc_fence_before();
