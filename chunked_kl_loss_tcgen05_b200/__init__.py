@@ -89,7 +89,7 @@ def load() -> ctypes.CDLL:
     lib.fckl_check.restype = ctypes.c_int
     lib.fckl_status_string.argtypes = [ctypes.c_int]
     lib.fckl_status_string.restype = ctypes.c_char_p
-    lib.fckl_profile_begin.argtypes = []
+    lib.fckl_profile_begin.argtypes = [ctypes.c_uint32]
     lib.fckl_profile_begin.restype = None
     lib.fckl_profile_end.argtypes = [ctypes.POINTER(FcklKernelStat), ctypes.c_int]
     lib.fckl_profile_end.restype = ctypes.c_int
@@ -135,8 +135,16 @@ def fckl_status_string(status: int) -> str:
     return load().fckl_status_string(int(status)).decode()
 
 
-def fckl_profile_begin() -> None:
-    load().fckl_profile_begin()
+KERNEL_KINDS = ("count_valid", "prep_teacher", "fwd_logits_lse", "merge_loss", "bwd_dlogits",
+                "dH_gemm", "dW_gemm", "finalize")
+
+
+def fckl_profile_begin(kinds=None) -> None:
+    """Start per-kernel event timing for the named kinds (None = all)."""
+    mask = 0
+    for k in (kinds or ()):
+        mask |= 1 << KERNEL_KINDS.index(k)
+    load().fckl_profile_begin(mask)
 
 
 def fckl_profile_end(max_stats: int = 16) -> list:

@@ -2,10 +2,11 @@
 // thread owns one accumulator row (TMEM lane) and walks the tile's 256
 // columns 32 at a time.
 //
-//   EpiLse      forward:  z = h W^T tile -> online (max, sum 2^(a - max)) of
-//               a = z log2(e) / T over the row's vocab tiles, plus a gather of
-//               z at the row's cached teacher ids.  Nothing of the tile is
-//               written; one (max, sum) partial per row per vocab segment.
+//   EpiLse      forward:  z = h W^T tile -> (max, sum 2^(a - max)) of
+//               a = z log2(e) / T over the tile's 256 vocab columns, plus a
+//               gather of z at the row's cached teacher ids that fall in the
+//               tile.  Nothing of the tile is written; one (max, sum) partial
+//               per row per vocab tile.
 //   EpiDlogits  backward: recomputed z tile -> q - p~ (0 for masked rows and
 //               for columns >= V), rounded once to bf16, staged in shared
 //               memory and TMA-stored to the chunk's dlogits block.
@@ -30,15 +31,6 @@
 
 namespace fckl {
 
-__device__ __forceinline__ int lower_bound_ids(const int* a, int n, int key) {
-  int lo = 0, hi = n;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (__ldg(a + mid) < key) lo = mid + 1; else hi = mid;
-  }
-  return lo;
-}
-
 // Warp-convergent TMEM load (tcgen05.ld must be executed by the whole warp).
 __device__ __forceinline__ void tmem_ld32_conv(uint32_t taddr, float (&v)[32]) {
   __syncwarp();
@@ -49,48 +41,41 @@ struct EpiLse {
   static constexpr uint32_t kSmemBytes = 0;
   static constexpr bool kUsesMapC = false;
   struct Params {
-    int rows_c;      // valid rows of this chunk
-    int V, K, Smax;
-    float scale2;    // log2(e) / T
-    const int* sid;  // [rows_c, K] ids sorted ascending (invalid ids -> INT_MAX)
-    float* zs;       // [rows_c, K] gathered z, same order as sid
-    float2* partials;  // [RB][Smax][128] (max, sum) in the log2 domain
+    int rows_c;               // valid rows of this chunk
+    int V, K, NT;
+    float scale2;             // log2(e) / T
+    const int* sid;           // [rows_c, K] ids sorted ascending (invalid ids -> INT_MAX)
+    const uint16_t* tstart;   // [rows_c, NT + 1] first sorted position of each vocab tile
+    float* zs;                // [rows_c, K] gathered z, same order as sid
+    float2* partials;         // [rows_c, NT] (max, sum) in the log2 domain
   };
-  struct State {
-    float m, s;
-    int cur, nid;
-  };
-  static __device__ void init(const Params&, State& st, uint8_t*, int) {
-    st.m = -INFINITY; st.s = 0.f; st.cur = 0; st.nid = INT_MAX;
-  }
-  static __device__ void tile(const Params& p, State& st, const Work& w, uint32_t taddr, int r,
+  struct State {};
+  static __device__ void init(const Params&, State&, uint8_t*, int) {}
+  static __device__ void tile(const Params& p, State&, const Work& w, uint32_t taddr, int r,
                               const CUtensorMap*, int, int) {
-    const int row = w.mb * BM + r;
+    const int row = w.m0 + r;
     const bool rv = row < p.rows_c;
     const int* rid = p.sid + (size_t)(rv ? row : 0) * p.K;
-    const int col0 = w.nb * BN;
-    if (w.seg_begin) {
-      st.m = -INFINITY;
-      st.s = 0.f;
-      if (rv) {
-        st.cur = lower_bound_ids(rid, p.K, col0);
-        st.nid = st.cur < p.K ? __ldg(rid + st.cur) : INT_MAX;
-      }
+    int cur = 0, nid = INT_MAX;
+    if (rv) {
+      cur = __ldg(p.tstart + (size_t)row * (p.NT + 1) + w.nt);
+      nid = cur < p.K ? __ldg(rid + cur) : INT_MAX;
     }
+    float m = -INFINITY, s = 0.f;
 #pragma unroll 1
     for (int c = 0; c < BN / 32; ++c) {
       float v[32];
       tmem_ld32_conv(taddr + (uint32_t)(c * 32), v);
       if (!rv) continue;
-      const int base = col0 + c * 32;
-      while (st.nid < base + 32) {  // gather z at cached ids in this 32-column slice
-        const int j = st.nid - base;
+      const int base = w.n0 + c * 32;
+      while (nid < base + 32) {  // gather z at cached ids in this 32-column slice
+        const int j = nid - base;
         float z = 0.f;
 #pragma unroll
         for (int jj = 0; jj < 32; ++jj) z = (jj == j) ? v[jj] : z;
-        p.zs[(size_t)row * p.K + st.cur] = z;
-        ++st.cur;
-        st.nid = st.cur < p.K ? __ldg(rid + st.cur) : INT_MAX;
+        p.zs[(size_t)row * p.K + cur] = z;
+        ++cur;
+        nid = cur < p.K ? __ldg(rid + cur) : INT_MAX;
       }
       float cm = -INFINITY;
       if (base + 32 <= p.V) {
@@ -104,15 +89,14 @@ struct EpiLse {
         }
       }
       if (cm == -INFINITY) continue;
-      const float nm = fmaxf(st.m, cm);
+      const float nm = fmaxf(m, cm);
       float acc = 0.f;
 #pragma unroll
       for (int j = 0; j < 32; ++j) acc += exp2f(v[j] - nm);
-      st.s = st.s * exp2f(st.m - nm) + acc;
-      st.m = nm;
+      s = s * exp2f(m - nm) + acc;
+      m = nm;
     }
-    if (w.seg_end && rv)
-      p.partials[((size_t)w.mb * p.Smax + w.split) * BM + r] = make_float2(st.m, st.s);
+    if (rv) p.partials[(size_t)row * p.NT + w.nt] = make_float2(m, s);
   }
   static __device__ void finish(const Params&, State&, int) {}
 };
@@ -143,12 +127,13 @@ struct EpiDlogits {
   static constexpr uint32_t kSmemBytes = 4 * 2 * 4096;
   static constexpr bool kUsesMapC = true;  // map C: dlogits [rows_c, V] bf16, box {64, 32}
   struct Params {
-    int rows_c, V, K;
-    float scale2;          // log2(e) / T
-    const float* lse2;     // [rows_c] log2-domain log-sum-exp of z / T
-    const int* sid;        // [rows_c, K] sorted ids
-    const float* sp;       // [rows_c, K] teacher probabilities, same order
-    const uint8_t* mask;   // chunk rows, or nullptr
+    int rows_c, V, K, NT;
+    float scale2;             // log2(e) / T
+    const float* lse2;        // [rows_c] log2-domain log-sum-exp of z / T
+    const int* sid;           // [rows_c, K] sorted ids
+    const uint16_t* tstart;   // [rows_c, NT + 1] first sorted position of each vocab tile
+    const float* sp;          // [rows_c, K] teacher probabilities, same order
+    const uint8_t* mask;      // chunk rows, or nullptr
   };
   struct State {
     int cur, nid, n;
@@ -184,16 +169,17 @@ struct EpiDlogits {
   }
   static __device__ void tile(const Params& p, State& st, const Work& w, uint32_t taddr, int r,
                               const CUtensorMap* mapC, int quarter, int lane) {
-    const int row = w.mb * BM + r;
+    const int row = w.m0 + r;
     const bool rv = row < p.rows_c;
     const bool keep = rv && (p.mask == nullptr || p.mask[row] != 0);
     const int* rid = p.sid + (size_t)(rv ? row : 0) * p.K;
     const float* rp = p.sp + (size_t)(rv ? row : 0) * p.K;
     const float lse = keep ? p.lse2[row] : 0.f;
-    const int col0 = w.nb * BN;
-    const int y = w.mb * BM + quarter * 32;
-    if (w.seg_begin && keep) {
-      st.cur = lower_bound_ids(rid, p.K, col0);
+    const int col0 = w.n0;
+    const int y = w.m0 + quarter * 32;
+    st.nid = INT_MAX;
+    if (keep) {
+      st.cur = __ldg(p.tstart + (size_t)row * (p.NT + 1) + w.nt);
       st.nid = st.cur < p.K ? __ldg(rid + st.cur) : INT_MAX;
     }
 #pragma unroll 1
@@ -283,9 +269,9 @@ struct EpiDH {
   }
   static __device__ void tile(const Params& p, State& st, const Work& w, uint32_t taddr, int,
                               const CUtensorMap* mapC, int quarter, int lane) {
-    const int y = w.mb * BM + quarter * 32;
-    stage_fp32_slices<true>(st.buf, st.n, taddr, st.alpha, mapC, w.nb * BN, p.H, y,
-                            y < p.rows_c, lane);
+    const int y = w.m0 + quarter * 32;
+    stage_fp32_slices<true>(st.buf, st.n, taddr, st.alpha, mapC, w.n0, p.H, y, y < p.rows_c,
+                            lane);
   }
   static __device__ void finish(const Params&, State&, int lane) {
     if (lane == 0) bulk_wait_all();
@@ -315,11 +301,11 @@ struct EpiDW {
   }
   static __device__ void tile(const Params& p, State& st, const Work& w, uint32_t taddr, int,
                               const CUtensorMap* mapC, int quarter, int lane) {
-    const int y = w.mb * BM + quarter * 32;
+    const int y = w.m0 + quarter * 32;
     if (p.accumulate)
-      stage_fp32_slices<true>(st.buf, st.n, taddr, st.alpha, mapC, w.nb * BN, p.H, y, y < p.V, lane);
+      stage_fp32_slices<true>(st.buf, st.n, taddr, st.alpha, mapC, w.n0, p.H, y, y < p.V, lane);
     else
-      stage_fp32_slices<false>(st.buf, st.n, taddr, st.alpha, mapC, w.nb * BN, p.H, y, y < p.V, lane);
+      stage_fp32_slices<false>(st.buf, st.n, taddr, st.alpha, mapC, w.n0, p.H, y, y < p.V, lane);
   }
   static __device__ void finish(const Params&, State&, int lane) {
     if (lane == 0) bulk_wait_all();

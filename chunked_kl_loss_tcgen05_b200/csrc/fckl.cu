@@ -23,15 +23,14 @@ namespace {
 
 constexpr size_t kAlign = 256;
 constexpr int kMaxDevices = 64;
-constexpr int kMaxGrid = 1024;  // partial-statistics slots are sized for at most this many CTAs
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
 
 struct Layout {
-  long long N, H, V, K, C, Vp, nchunks, RBmax;
-  size_t off_rowloss, off_sid, off_sp, off_zs, off_plogp, off_lse2, off_part, off_dlog, total;
-  size_t part_slots;  // float2 entries reserved for partial statistics
+  long long N, H, V, K, C, Vp, nchunks, NT;
+  size_t off_rowloss, off_sid, off_sp, off_zs, off_tstart, off_plogp, off_lse2, off_part,
+      off_dlog, total;
 };
 
 bool valid_problem(const fckl_problem* p) {
@@ -64,17 +63,17 @@ Layout make_layout(const fckl_problem* p) {
   L.Vp = (long long)align_up((size_t)p->V, 8);
   L.C = resolve_chunk(p);
   L.nchunks = cdiv(L.N, L.C);
-  L.RBmax = cdiv(L.C, BM);
+  L.NT = cdiv(L.V, BN);
   size_t off = align_up(sizeof(DeviceCtl), kAlign);
   auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, kAlign); return o; };
   L.off_rowloss = take((size_t)L.N * 4);
   L.off_sid = take((size_t)L.C * L.K * 4);
   L.off_sp = take((size_t)L.C * L.K * 4);
   L.off_zs = take((size_t)L.C * L.K * 4);
+  L.off_tstart = take((size_t)L.C * (L.NT + 1) * 2);
   L.off_plogp = take((size_t)L.C * 4);
   L.off_lse2 = take((size_t)L.C * 4);
-  L.part_slots = (size_t)(kMaxGrid + 2 * L.RBmax) * BM;
-  L.off_part = take(L.part_slots * sizeof(float2));
+  L.off_part = take((size_t)L.C * L.NT * sizeof(float2));
   L.off_dlog = take((size_t)L.C * L.Vp * 2);
   L.total = off;
   return L;
@@ -126,11 +125,11 @@ struct DeviceInfo {
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
 
-template <class Sched, class Epi, bool A_MN, bool B_MN>
+template <class Epi, bool A_MN, bool B_MN>
 bool set_smem_attr() {
-  return cudaFuncSetAttribute(gemm_kernel<Sched, Epi, A_MN, B_MN>,
+  return cudaFuncSetAttribute(gemm_pair_kernel<Epi, A_MN, B_MN>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)gemm_smem_bytes<Epi>()) == cudaSuccess;
+                              (int)pair_smem_bytes<Epi>()) == cudaSuccess;
 }
 
 const DeviceInfo* device_info() {
@@ -146,12 +145,9 @@ const DeviceInfo* device_info() {
     cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
     d.ok = major == 10 && minor == 0 && d.sms > 0;
     if (d.ok) {
-      d.ok = set_smem_attr<SchedLinear, EpiLse, false, false>() &&
-             set_smem_attr<SchedLinear, EpiDlogits, false, false>() &&
-             set_smem_attr<SchedSplitK, EpiDH, false, true>() &&
-             set_smem_attr<SchedTiles, EpiDW, true, true>();
+      d.ok = set_smem_attr<EpiLse, false, false>() && set_smem_attr<EpiDlogits, false, false>() &&
+             set_smem_attr<EpiDH, false, true>() && set_smem_attr<EpiDW, true, true>();
     }
-    d.sms = std::min(d.sms, kMaxGrid);
   }
   return &d;
 }
@@ -181,6 +177,7 @@ struct ProfRec {
 };
 struct Profiler {
   bool on = false;
+  uint32_t mask = 0xFFFFFFFFu;
   std::vector<ProfRec> recs;
   std::vector<cudaEvent_t> pool;
   size_t used = 0;
@@ -201,7 +198,8 @@ struct ProfScope {
   double flops, bytes;
   cudaEvent_t a = nullptr;
   ProfScope(int k, cudaStream_t s, double f, double b) : kind(k), st(s), flops(f), bytes(b) {
-    if (g_prof.on && (a = g_prof.next()) != nullptr) cudaEventRecord(a, st);
+    if (g_prof.on && ((g_prof.mask >> k) & 1u) && (a = g_prof.next()) != nullptr)
+      cudaEventRecord(a, st);
   }
   ~ProfScope() {
     if (!g_prof.on || a == nullptr) return;
@@ -212,27 +210,19 @@ struct ProfScope {
   }
 };
 
-// Split-K factor for dH: minimise waves * (k-blocks per unit + fixed cost).
-int choose_split(long long tiles, long long KB, int sms) {
+// Split-K factor for dH: minimise waves * (k-blocks per unit + fixed cost),
+// with `slots` CTA pairs working at once.
+int choose_split(long long tiles, long long KB, int slots) {
   int best = 1;
   double best_cost = 1e300;
   const long long smax = std::min<long long>(KB, 512);
   for (long long S = 1; S <= smax; ++S) {
     const long long units = tiles * S;
-    const double waves = (double)cdiv(units, sms);
+    const double waves = (double)cdiv(units, slots);
     const double cost = waves * ((double)cdiv(KB, S) + 6.0);
     if (cost < best_cost - 1e-9) { best_cost = cost; best = (int)S; }
   }
   return best;
-}
-
-int max_splits(long long RB, long long NT, long long total, long long G) {
-  long long m = 1;
-  for (long long rb = 0; rb < RB; ++rb) {
-    const long long n = lin_owner(rb * NT + NT - 1, total, G) - lin_owner(rb * NT, total, G) + 1;
-    m = std::max(m, n);
-  }
-  return (int)m;
 }
 
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -263,6 +253,7 @@ fckl_status run(bool bwd, const fckl_problem* prob, const void* hidden, const vo
   int* sid = reinterpret_cast<int*>(ws + L.off_sid);
   float* sp = reinterpret_cast<float*>(ws + L.off_sp);
   float* zs = reinterpret_cast<float*>(ws + L.off_zs);
+  uint16_t* tstart = reinterpret_cast<uint16_t*>(ws + L.off_tstart);
   float* plogp = reinterpret_cast<float*>(ws + L.off_plogp);
   float* lse2 = reinterpret_cast<float*>(ws + L.off_lse2);
   float2* part = reinterpret_cast<float2*>(ws + L.off_part);
@@ -280,101 +271,96 @@ fckl_status run(bool bwd, const fckl_problem* prob, const void* hidden, const vo
   }
 
   CUtensorMap mapW_k, mapW_mn, mapdW;
-  if (!make_map(&mapW_k, W, L.H, L.V, L.H * 2, BK, BN)) return FCKL_ERR_CUDA;
+  if (!make_map(&mapW_k, W, L.H, L.V, L.H * 2, BK, BN / 2)) return FCKL_ERR_CUDA;
   if (bwd && !make_map(&mapW_mn, W, L.H, L.V, L.H * 2, 64, BK)) return FCKL_ERR_CUDA;
   if (bwd && !make_map(&mapdW, dW, L.H, L.V, L.H * 4, 32, 32, true)) return FCKL_ERR_CUDA;
 
-  const long long NT = cdiv(L.V, BN);
+  const int pairs = std::max(1, dev->sms / 2);  // CTA pairs that run at once
+  const long long NT = L.NT;
   const long long KBh = cdiv(L.H, BK);
+  const long long NTh = cdiv(L.H, BN);
+  const long long KBv = cdiv(L.V, BK);
+  auto grid_for = [&](long long units) { return (int)(2 * std::min<long long>(pairs, units)); };
   for (long long c = 0; c < L.nchunks; ++c) {
     const long long row0 = c * L.C;
     const int rows = (int)std::min(L.C, L.N - row0);
-    const long long RB = cdiv(rows, BM);
+    const long long MT = cdiv(rows, PM);
     const uint8_t* mask_c = row_mask ? row_mask + row0 : nullptr;
     const void* h_c = static_cast<const uint8_t*>(hidden) + (size_t)row0 * L.H * 2;
     const int row_blocks = (int)cdiv(rows, ROW_WARPS);
 
     {
-      ProfScope ps(K_PREP, st, 0.0, (double)rows * K * 20.0 + rows * 5.0);
+      ProfScope ps(K_PREP, st, 0.0, (double)rows * K * 20.0 + rows * (NT + 1) * 2.0);
       k_prep_teacher<<<row_blocks, ROW_WARPS * 32, 0, st>>>(
-          topk_idx + row0 * K, topk_logit + row0 * K, mask_c, rows, K, V, invT, sid, sp, zs,
-          plogp, ctl);
+          topk_idx + row0 * K, topk_logit + row0 * K, mask_c, rows, K, V, (int)NT, invT, sid, sp,
+          zs, tstart, plogp, ctl);
     }
 
     CUtensorMap mapH_k;
-    if (!make_map(&mapH_k, h_c, L.H, rows, L.H * 2, BK, BM)) return FCKL_ERR_CUDA;
+    if (!make_map(&mapH_k, h_c, L.H, rows, L.H * 2, BK, CM)) return FCKL_ERR_CUDA;
 
-    const long long total = RB * NT;
-    const int G = (int)std::min<long long>(dev->sms, total);
-    const int Smax = max_splits(RB, NT, total, G);
-    if ((size_t)RB * Smax * BM > L.part_slots) return FCKL_ERR_UNSUPPORTED;
-    SchedArgs sa_lin{total, (int)NT, (int)KBh, 1, 0};
-
-    EpiLse::Params pf{rows, V, K, Smax, scale2, sid, zs, part};
+    // Forward: z = h W^T tiles, vocab-major units so concurrent pairs share W tiles.
+    SchedArgs sa_v{MT * NT, SCHED_VOCAB_MAJOR, (int)MT, (int)NT, (int)KBh, 1, 0};
+    const int Gv = grid_for(MT * NT);
+    EpiLse::Params pf{rows, V, K, (int)NT, scale2, sid, tstart, zs, part};
     CtlArgs ca_f = ca;
     ca_f.debug_skip_commit = (c == 0) ? ca.debug_skip_commit : 0;
     const double gemm_flops = 2.0 * rows * (double)L.V * (double)L.H;
     {
-      ProfScope ps(K_FWD, st, gemm_flops, 2.0 * (rows + (double)L.V) * L.H + rows * K * 4.0);
-      gemm_kernel<SchedLinear, EpiLse, false, false>
-          <<<G, GEMM_THREADS, gemm_smem_bytes<EpiLse>(), st>>>(mapH_k, mapW_k, mapW_k, pf,
-                                                               sa_lin, ca_f);
+      ProfScope ps(K_FWD, st, gemm_flops, 2.0 * (rows + (double)L.V) * L.H + rows * NT * 8.0);
+      gemm_pair_kernel<EpiLse, false, false>
+          <<<Gv, GEMM_THREADS, pair_smem_bytes<EpiLse>(), st>>>(mapH_k, mapW_k, mapW_k, pf, sa_v,
+                                                                ca_f);
     }
-
     {
-      ProfScope ps(K_MERGE, st, 0.0, (double)rows * K * 8.0 + rows * 13.0);
-      k_merge_loss<<<row_blocks, ROW_WARPS * 32, 0, st>>>(part, Smax, (int)NT, total, G, rows,
-                                                           K, invT, zs, sp, plogp, mask_c, lse2,
-                                                           rl + row0);
+      ProfScope ps(K_MERGE, st, 0.0, (double)rows * K * 8.0 + rows * NT * 8.0 + rows * 13.0);
+      k_merge_loss<<<row_blocks, ROW_WARPS * 32, 0, st>>>(part, (int)NT, rows, K, invT, zs, sp,
+                                                           plogp, mask_c, lse2, rl + row0);
     }
     if (!bwd) continue;
 
-    EpiDlogits::Params pb{rows, V, K, scale2, lse2, sid, sp, mask_c};
+    // Backward 1: recompute the tiles and form bf16 dlogits = q - p~.
+    EpiDlogits::Params pb{rows, V, K, (int)NT, scale2, lse2, sid, tstart, sp, mask_c};
     CUtensorMap mapD_st;
     if (!make_map(&mapD_st, dlog, L.V, rows, L.Vp * 2, 64, 32)) return FCKL_ERR_CUDA;
     {
       ProfScope ps(K_BWD, st, gemm_flops, 2.0 * (rows + (double)L.V) * L.H + 2.0 * rows * L.V);
-      gemm_kernel<SchedLinear, EpiDlogits, false, false>
-          <<<G, GEMM_THREADS, gemm_smem_bytes<EpiDlogits>(), st>>>(mapH_k, mapW_k, mapD_st, pb,
-                                                                   sa_lin, ca);
+      gemm_pair_kernel<EpiDlogits, false, false>
+          <<<Gv, GEMM_THREADS, pair_smem_bytes<EpiDlogits>(), st>>>(mapH_k, mapW_k, mapD_st, pb,
+                                                                    sa_v, ca);
     }
 
-    // dH[rows] = alpha * dlogits W : A = dlogits (K-major), B = W (MN-major).
+    // Backward 2: dH[rows] = alpha * dlogits W; A = dlogits (K-major), B = W (MN-major).
     if (cudaMemsetAsync(dH + row0 * L.H, 0, (size_t)rows * L.H * 4, st) != cudaSuccess)
       return FCKL_ERR_CUDA;
-    CUtensorMap mapD_k, mapD_mn, mapH_mn;
-    if (!make_map(&mapD_k, dlog, L.V, rows, L.Vp * 2, BK, BM)) return FCKL_ERR_CUDA;
-    const long long NTh = cdiv(L.H, BN);
-    const long long tiles_h = RB * NTh;
-    const long long KBv = cdiv(L.V, BK);
-    const int S = choose_split(tiles_h, KBv, dev->sms);
-    SchedArgs sa_dh{tiles_h * S, (int)NTh, (int)KBv, S, (int)tiles_h};
-    const int Gh = (int)std::min<long long>(dev->sms, tiles_h * S);
-    EpiDH::Params ph{rows, H, invT, ctl};
-    CUtensorMap mapdH;
+    CUtensorMap mapD_k, mapD_mn, mapH_mn, mapdH;
+    if (!make_map(&mapD_k, dlog, L.V, rows, L.Vp * 2, BK, CM)) return FCKL_ERR_CUDA;
     if (!make_map(&mapdH, dH + row0 * L.H, L.H, rows, L.H * 4, 32, 32, true)) return FCKL_ERR_CUDA;
+    const long long tiles_h = MT * NTh;
+    const int S = choose_split(tiles_h, KBv, pairs);
+    SchedArgs sa_h{tiles_h * S, SCHED_SPLIT_K, (int)MT, (int)NTh, (int)KBv, S, (int)tiles_h};
+    EpiDH::Params ph{rows, H, invT, ctl};
     {
       ProfScope ps(K_DH, st, gemm_flops,
                    2.0 * rows * (double)L.V + 2.0 * (double)L.V * L.H + 4.0 * rows * L.H);
-      gemm_kernel<SchedSplitK, EpiDH, false, true>
-          <<<Gh, GEMM_THREADS, gemm_smem_bytes<EpiDH>(), st>>>(mapD_k, mapW_mn, mapdH, ph, sa_dh,
-                                                               ca);
+      gemm_pair_kernel<EpiDH, false, true>
+          <<<grid_for(tiles_h * S), GEMM_THREADS, pair_smem_bytes<EpiDH>(), st>>>(
+              mapD_k, mapW_mn, mapdH, ph, sa_h, ca);
     }
 
-    // dW (+)= alpha * dlogits^T h : A = dlogits^T (MN-major), B = h (MN-major).
+    // Backward 3: dW (+)= alpha * dlogits^T h; A = dlogits^T, B = h (both MN-major).
     if (!make_map(&mapD_mn, dlog, L.V, rows, L.Vp * 2, 64, BK)) return FCKL_ERR_CUDA;
     if (!make_map(&mapH_mn, h_c, L.H, rows, L.H * 2, 64, BK)) return FCKL_ERR_CUDA;
-    const long long tiles_w = cdiv(L.V, BM) * NTh;
-    SchedArgs sa_dw{tiles_w, (int)NTh, (int)cdiv(rows, BK), 1, (int)tiles_w};
-    const int Gw = (int)std::min<long long>(dev->sms, tiles_w);
+    const long long tiles_w = cdiv(L.V, PM) * NTh;
+    SchedArgs sa_w{tiles_w, SCHED_TILES, 0, (int)NTh, (int)cdiv(rows, BK), 1, (int)tiles_w};
     EpiDW::Params pw{V, H, invT, c > 0 ? 1 : 0, ctl};
     {
       ProfScope ps(K_DW, st, gemm_flops,
                    2.0 * rows * (double)L.V + 2.0 * rows * L.H +
                        (c > 0 ? 8.0 : 4.0) * (double)L.V * L.H);
-      gemm_kernel<SchedTiles, EpiDW, true, true>
-          <<<Gw, GEMM_THREADS, gemm_smem_bytes<EpiDW>(), st>>>(mapD_mn, mapH_mn, mapdW, pw, sa_dw,
-                                                               ca);
+      gemm_pair_kernel<EpiDW, true, true>
+          <<<grid_for(tiles_w), GEMM_THREADS, pair_smem_bytes<EpiDW>(), st>>>(
+              mapD_mn, mapH_mn, mapdW, pw, sa_w, ca);
     }
   }
   {
@@ -428,8 +414,9 @@ fckl_status fckl_check(void* workspace, void* stream) {
   return FCKL_OK;
 }
 
-void fckl_profile_begin(void) {
+void fckl_profile_begin(uint32_t kind_mask) {
   g_prof.on = true;
+  g_prof.mask = kind_mask ? kind_mask : 0xFFFFFFFFu;
   g_prof.recs.clear();
   g_prof.used = 0;
 }

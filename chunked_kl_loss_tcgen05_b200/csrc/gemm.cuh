@@ -1,42 +1,60 @@
 // Persistent, warp-specialised tcgen05 GEMM core shared by the four GEMMs of
-// the fused chunked KL loss.
+// the fused chunked KL loss, run on CTA pairs (clusters of 2).
 //
-//   warp 0      TMA producer: one elected thread streams 64-wide k-blocks of A
-//               and B into a ring of shared-memory stages (128B swizzle).
-//   warp 1      allocates 512 TMEM columns (two 128x256 fp32 accumulators) and
-//               one elected thread issues tcgen05.mma (M=128, N=256, K=16).
-//   warps 2-5   epilogue: tcgen05.ld the finished accumulator (thread = row),
-//               run the kernel-specific epilogue, release the accumulator.
+// One work unit is a 256 x 256 output tile computed by a CTA pair with
+// tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16 per instruction):
+//   * CTA r (r = 0, 1) stages rows [128 r, +128) of A and columns
+//     [128 r, +128) of B in its own shared memory (128-byte swizzle); no
+//     multicast copies are used;
+//   * the even CTA's single MMA thread issues the MMAs for the pair; each CTA's
+//     TMEM receives the fp32 accumulator of its own 128 rows x 256 columns;
+//   * each CTA's epilogue reads its own TMEM.
 //
-// Double-buffered accumulators let the epilogue of tile i overlap the
-// main loop of tile i+1.  Every wait is bounded (see ptx.cuh).
+// Warp roles in every CTA (192 threads):
+//   warp 0      TMA producer (one thread): waits for a free stage, loads this
+//               CTA's A and B halves; the completion of both CTAs' copies is
+//               counted on the even CTA's "full" barrier.
+//   warp 1      allocates 512 TMEM columns (two accumulators) for the pair; in
+//               the even CTA one thread issues the MMAs, frees stages in both
+//               CTAs and announces finished accumulators to both CTAs with
+//               multicast tcgen05.commit.
+//   warps 2-5   epilogue: tcgen05.ld (thread = row), kernel-specific epilogue,
+//               then release the accumulator on the even CTA's barrier.
+// Double-buffered accumulators overlap the epilogue of one tile with the main
+// loop of the next.  Every wait is bounded (see ptx.cuh).
 //
-// Operand majors (bf16, row-major global tensors):
+// Operand majors (bf16, row-major global tensors), per CTA and stage:
 //   A K-major  : A[m, k] contiguous in k  -> TMA box {64 k, 128 m}
 //   A MN-major : A[m, k] contiguous in m  -> two TMA boxes {64 m, 64 k}
-//   B K-major  : B[n, k] contiguous in k  -> TMA box {64 k, 256 n}
-//   B MN-major : B[n, k] contiguous in n  -> four TMA boxes {64 n, 64 k}
+//   B K-major  : B[n, k] contiguous in k  -> TMA box {64 k, 128 n}
+//   B MN-major : B[n, k] contiguous in n  -> two TMA boxes {64 n, 64 k}
 #pragma once
 
 #include "ptx.cuh"
 
 namespace fckl {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
-constexpr int BK = 64;
-constexpr int STAGES = 4;
-constexpr uint32_t A_STAGE_BYTES = BM * BK * 2;  // 16 KB
-constexpr uint32_t B_STAGE_BYTES = BN * BK * 2;  // 32 KB
-constexpr uint32_t STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
+constexpr int PM = 256;  // rows of a pair tile
+constexpr int CM = 128;  // rows per CTA
+constexpr int BN = 256;  // columns of a tile
+constexpr int BK = 64;   // k-block
+constexpr uint32_t A_HALF_BYTES = CM * BK * 2;        // 16 KB
+constexpr uint32_t B_HALF_BYTES = (BN / 2) * BK * 2;  // 16 KB
+constexpr uint32_t PSTAGE_BYTES = A_HALF_BYTES + B_HALF_BYTES;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int GEMM_THREADS = 192;
+constexpr size_t SMEM_LIMIT = 232448;  // opt-in dynamic shared memory per CTA on sm_100
+
 // Dynamic shared memory: 1 KB alignment slack, the operand stages, the
-// epilogue's staging area (Epi::kSmemBytes, split evenly over the 4 epilogue
-// warps) and 256 bytes of barriers.
+// epilogue's staging area (Epi::kSmemBytes, split over the 4 epilogue warps)
+// and 256 bytes of barriers.  As many stages as fit.
 template <class Epi>
-constexpr size_t gemm_smem_bytes() {
-  return 1024 + (size_t)STAGES * STAGE_BYTES + Epi::kSmemBytes + 256;
+__host__ __device__ constexpr int pair_stages() {
+  return (int)((SMEM_LIMIT - 1024 - 256 - Epi::kSmemBytes) / PSTAGE_BYTES);
+}
+template <class Epi>
+__host__ __device__ constexpr size_t pair_smem_bytes() {
+  return 1024 + (size_t)pair_stages<Epi>() * PSTAGE_BYTES + Epi::kSmemBytes + 256;
 }
 
 // Wait-site codes recorded on timeout (diagnostics only).
@@ -46,89 +64,54 @@ enum : uint32_t {
 };
 
 struct Work {
-  int mb, nb;      // tile coordinates: rows [mb*128, +128), cols [nb*256, +256)
-  int kb0, kb1;    // k-blocks [kb0, kb1) of 64
-  int split;       // partial-result slot (vocab-split kernels)
-  bool seg_begin;  // first tile of a run of consecutive vocab tiles of one row block
-  bool seg_end;    // last tile of that run
+  int mt, nt;    // pair tile: rows [mt*256, +256), columns [nt*256, +256)
+  int kb0, kb1;  // k-blocks [kb0, kb1) of 64
+  int m0, n0;    // this CTA's first row (mt*256 + 128*rank) and the first column
 };
 
-// Scheduling arguments (one struct for every scheduler).
+enum SchedKind : int {
+  SCHED_VOCAB_MAJOR = 0,  // units (vocab tile nt, row tile mt), mt fastest; full K
+  SCHED_SPLIT_K = 1,      // units (k segment, output tile), k segment slowest
+  SCHED_TILES = 2,        // units (mt, nt), nt fastest; full K
+};
+
 struct SchedArgs {
-  long long total;  // linear schedule: RB * NT tiles; unit schedules: number of units
-  int NT;           // tiles along n per row block (linear) / n tiles (unit schedules)
+  long long total;  // number of units
+  int kind;
+  int MT;           // row tiles (SCHED_VOCAB_MAJOR)
+  int NT;           // column tiles (SCHED_SPLIT_K, SCHED_TILES)
   int KB;           // k-blocks of the full reduction
-  int S;            // split-K factor (split-K schedule)
-  int tiles;        // output tiles (split-K schedule)
+  int S;            // split-K factor
+  int tiles;        // output tiles (SCHED_SPLIT_K)
 };
 
-// Linear schedule over (row block, vocab tile), row-block-major; CTA i owns the
-// contiguous range [i*T/G, (i+1)*T/G).  Tiles of one row block that fall in one
-// CTA form a segment, whose per-row partial statistics land in slot `split`.
-__host__ __device__ inline long long lin_begin(long long i, long long total, long long G) {
-  return i * total / G;
-}
-// The CTA whose range contains tile x.
-__host__ __device__ inline long long lin_owner(long long x, long long total, long long G) {
-  return ((x + 1) * G + total - 1) / total - 1;
-}
-
-struct SchedLinear {
-  long long t, t_beg, t_end, total;
-  int NT, KB, G, cta;
-  __device__ void init(const SchedArgs& a, int cta_, int G_) {
-    total = a.total; NT = a.NT; KB = a.KB; G = G_; cta = cta_;
-    t_beg = lin_begin(cta, total, G);
-    t_end = lin_begin(cta + 1, total, G);
-    t = t_beg;
+// Cluster c of G takes units c, c+G, c+2G, ...  In every order above, the
+// clusters running at the same moment touch a narrow band of the streamed
+// operand, so it is read from DRAM about once and reused from L2.
+struct PairSched {
+  long long u;
+  SchedArgs a;
+  int G;
+  __device__ void init(const SchedArgs& args, int cluster, int nclusters) {
+    a = args; G = nclusters; u = cluster;
   }
   __device__ bool next(Work& w) {
-    if (t >= t_end) return false;
-    const int rb = (int)(t / NT);
-    const int vt = (int)(t - (long long)rb * NT);
-    w.mb = rb; w.nb = vt; w.kb0 = 0; w.kb1 = KB;
-    w.seg_begin = (t == t_beg) || (vt == 0);
-    w.seg_end = (t + 1 == t_end) || (vt == NT - 1);
-    w.split = cta - (int)lin_owner((long long)rb * NT, total, G);
-    ++t;
-    return true;
-  }
-};
-
-// Split-K over the reduction dimension: units ordered k-segment-major so that
-// all CTAs read the same k-slab of both operands at about the same time (the
-// slab stays in L2).  CTA i takes units i, i+G, i+2G, ...
-struct SchedSplitK {
-  long long u, total;
-  int G, tiles, NT, KB, S;
-  __device__ void init(const SchedArgs& a, int cta, int G_) {
-    total = a.total; tiles = a.tiles; NT = a.NT; KB = a.KB; S = a.S; G = G_; u = cta;
-  }
-  __device__ bool next(Work& w) {
-    if (u >= total) return false;
-    const int ks = (int)(u / tiles);
-    const int tile = (int)(u - (long long)ks * tiles);
-    w.mb = tile / NT; w.nb = tile - w.mb * NT;
-    w.kb0 = (int)((long long)ks * KB / S);
-    w.kb1 = (int)((long long)(ks + 1) * KB / S);
-    w.split = ks; w.seg_begin = true; w.seg_end = true;
-    u += G;
-    return true;
-  }
-};
-
-// Whole-K output tiles, CTA i takes tiles i, i+G, ...; consecutive tiles share
-// the same m block (same A panel).
-struct SchedTiles {
-  long long u, total;
-  int G, NT, KB;
-  __device__ void init(const SchedArgs& a, int cta, int G_) {
-    total = a.total; NT = a.NT; KB = a.KB; G = G_; u = cta;
-  }
-  __device__ bool next(Work& w) {
-    if (u >= total) return false;
-    w.mb = (int)(u / NT); w.nb = (int)(u - (long long)w.mb * NT);
-    w.kb0 = 0; w.kb1 = KB; w.split = 0; w.seg_begin = true; w.seg_end = true;
+    if (u >= a.total) return false;
+    if (a.kind == SCHED_VOCAB_MAJOR) {
+      w.nt = (int)(u / a.MT);
+      w.mt = (int)(u - (long long)w.nt * a.MT);
+      w.kb0 = 0; w.kb1 = a.KB;
+    } else if (a.kind == SCHED_SPLIT_K) {
+      const int ks = (int)(u / a.tiles);
+      const int tile = (int)(u - (long long)ks * a.tiles);
+      w.mt = tile / a.NT; w.nt = tile - w.mt * a.NT;
+      w.kb0 = (int)((long long)ks * a.KB / a.S);
+      w.kb1 = (int)((long long)(ks + 1) * a.KB / a.S);
+    } else {
+      w.mt = (int)(u / a.NT);
+      w.nt = (int)(u - (long long)w.mt * a.NT);
+      w.kb0 = 0; w.kb1 = a.KB;
+    }
     u += G;
     return true;
   }
@@ -140,28 +123,34 @@ struct CtlArgs {
   int debug_skip_commit;  // >0: the MMA thread omits its first accumulator-ready commit
 };
 
-template <class Sched, class Epi, bool A_MN, bool B_MN>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const __grid_constant__ CUtensorMap tmC, const typename Epi::Params ep,
-                const SchedArgs sa, const CtlArgs ca) {
+template <class Epi, bool A_MN, bool B_MN>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                     const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmC, const typename Epi::Params ep,
+                     const SchedArgs sa, const CtlArgs ca) {
+  constexpr int STAGES = pair_stages<Epi>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* sA = smem;
-  uint8_t* sB = smem + STAGES * A_STAGE_BYTES;
-  uint8_t* sEpi = smem + STAGES * STAGE_BYTES;  // 1 KB aligned
+  uint8_t* sA = smem;                                  // [STAGES][16 KB]
+  uint8_t* sB = smem + STAGES * A_HALF_BYTES;          // [STAGES][16 KB]
+  uint8_t* sEpi = smem + STAGES * PSTAGE_BYTES;        // 1 KB aligned
   uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + Epi::kSmemBytes);
-  uint64_t* full = bars;                // [STAGES]  TMA -> MMA
-  uint64_t* empty = bars + STAGES;      // [STAGES]  MMA -> TMA
-  uint64_t* tfull = bars + 2 * STAGES;  // [2]       MMA -> epilogue
-  uint64_t* tempty = tfull + 2;         // [2]       epilogue -> MMA
-  uint64_t* drain = tempty + 2;         // [1]       MMA drain at exit
+  uint64_t* full = bars;                 // [STAGES]  TMA (both CTAs) -> MMA   (even CTA's used)
+  uint64_t* empty = bars + STAGES;       // [STAGES]  MMA -> TMA               (each CTA's own)
+  uint64_t* tfull = bars + 2 * STAGES;   // [2]       MMA -> epilogue          (each CTA's own)
+  uint64_t* tempty = tfull + 2;          // [2]       epilogues -> MMA         (even CTA's used)
+  uint64_t* drain = tempty + 2;          // [1]       MMA drain at exit        (even CTA's used)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   uint32_t* abort_flag = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cluster = blockIdx.x >> 1;
+  const int nclusters = gridDim.x >> 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -170,7 +159,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(smem_u32(&tfull[a]), 1);
-      mbar_init(smem_u32(&tempty[a]), 4);
+      mbar_init(smem_u32(&tempty[a]), 8);  // 4 epilogue warps in each CTA of the pair
     }
     mbar_init(smem_u32(drain), 1);
     *abort_flag = 0u;
@@ -180,11 +169,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     if (Epi::kUsesMapC) tma_prefetch_desc(&tmC);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();  // barriers of both CTAs initialised before any remote use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const WaitCtx wc{ca.timeout_ns, ca.ctl, abort_flag};
@@ -192,58 +182,67 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      Sched sch;
-      sch.init(sa, blockIdx.x, gridDim.x);
+      PairSched sch;
+      sch.init(sa, cluster, nclusters);
       Work w;
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t armed = 0;  // bit s: stage s has been armed at least once
-      uint32_t last_parity = 0;  // bit s: parity of the last armed phase of stage s
+      uint32_t armed = 0, last_parity = 0;  // even CTA: which full phases it armed
       bool ok = true;
       while (ok && sch.next(w)) {
+        const int a_row = w.mt * PM + (int)rank * CM;
+        const int b_col = w.nt * BN + (int)rank * (BN / 2);
         for (int kb = w.kb0; kb < w.kb1; ++kb) {
           if (!wait_phase(smem_u32(&empty[stage]), phase ^ 1u, wc, SITE_PROD_EMPTY)) {
             ok = false;
             break;
           }
-          const uint32_t fb = smem_u32(&full[stage]);
-          mbar_arrive_expect_tx(fb, STAGE_BYTES);
-          armed |= 1u << stage;
-          last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
-          const uint32_t a_dst = smem_u32(sA + stage * A_STAGE_BYTES);
-          const uint32_t b_dst = smem_u32(sB + stage * B_STAGE_BYTES);
+          const uint32_t fb_local = smem_u32(&full[stage]);
+          if (leader) {
+            mbar_arrive_expect_tx(fb_local, 2 * PSTAGE_BYTES);
+            armed |= 1u << stage;
+            last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+          }
+          const uint32_t fb = mapa_shared(fb_local, 0);
+          const uint32_t a_dst = smem_u32(sA + stage * A_HALF_BYTES);
+          const uint32_t b_dst = smem_u32(sB + stage * B_HALF_BYTES);
           const int k0 = kb * BK;
           if (!A_MN) {
-            tma_load_2d(a_dst, &tmA, fb, k0, w.mb * BM);
+            tma_load_2d_pair(a_dst, &tmA, fb, k0, a_row);
           } else {
-            tma_load_2d(a_dst, &tmA, fb, w.mb * BM, k0);
-            tma_load_2d(a_dst + 8192, &tmA, fb, w.mb * BM + 64, k0);
+            tma_load_2d_pair(a_dst, &tmA, fb, a_row, k0);
+            tma_load_2d_pair(a_dst + 8192, &tmA, fb, a_row + 64, k0);
           }
           if (!B_MN) {
-            tma_load_2d(b_dst, &tmB, fb, k0, w.nb * BN);
+            tma_load_2d_pair(b_dst, &tmB, fb, k0, b_col);
           } else {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) tma_load_2d(b_dst + j * 8192, &tmB, fb, w.nb * BN + 64 * j, k0);
+            tma_load_2d_pair(b_dst, &tmB, fb, b_col, k0);
+            tma_load_2d_pair(b_dst + 8192, &tmB, fb, b_col + 64, k0);
           }
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
-      // Let every copy this thread started land before the CTA can exit.
-      for (int s = 0; s < STAGES; ++s)
-        if (armed & (1u << s)) drain_phase(smem_u32(&full[s]), (last_parity >> s) & 1u, wc, SITE_DRAIN_TMA);
+      if (leader) {
+        // Every copy counted on an armed phase has landed before the pair can exit.
+        for (int s = 0; s < STAGES; ++s)
+          if (armed & (1u << s))
+            drain_phase(smem_u32(&full[s]), (last_parity >> s) & 1u, wc, SITE_DRAIN_TMA);
+      } else if (!ok) {
+        __nanosleep(20000);  // aborted: give copies already issued time to land
+      }
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      Sched sch;
-      sch.init(sa, blockIdx.x, gridDim.x);
+    if (leader && lane == 0) {
+      PairSched sch;
+      sch.init(sa, cluster, nclusters);
       Work w;
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
-      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, A_MN, B_MN);
+      constexpr uint32_t idesc = idesc_bf16_f32(PM, BN, A_MN, B_MN);
       bool ok = true;
       int skip = ca.debug_skip_commit;
       while (ok && sch.next(w)) {
@@ -256,30 +255,30 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a_base = smem_u32(sA + stage * A_STAGE_BYTES);
-          const uint32_t b_base = smem_u32(sB + stage * B_STAGE_BYTES);
+          const uint32_t a_base = smem_u32(sA + stage * A_HALF_BYTES);
+          const uint32_t b_base = smem_u32(sB + stage * B_HALF_BYTES);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             const uint64_t ad = A_MN ? sw128_desc(a_base + k * 2048, 8192, 1024)
                                      : sw128_desc(a_base + k * 32, 16, 1024);
             const uint64_t bd = B_MN ? sw128_desc(b_base + k * 2048, 8192, 1024)
                                      : sw128_desc(b_base + k * 32, 16, 1024);
-            umma_bf16(d_tmem, ad, bd, idesc, (kb > w.kb0 || k > 0) ? 1u : 0u);
+            umma_bf16_pair(d_tmem, ad, bd, idesc, (kb > w.kb0 || k > 0) ? 1u : 0u);
           }
-          umma_commit(smem_u32(&empty[stage]));  // frees the stage once these MMAs finish
+          umma_commit_pair(smem_u32(&empty[stage]), 0x3);  // frees the stage in both CTAs
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
         if (skip > 0) {
           --skip;  // fault-injection knob: this accumulator is never announced
         } else {
-          umma_commit(smem_u32(&tfull[acc]));
+          umma_commit_pair(smem_u32(&tfull[acc]), 0x3);
         }
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
-      // Wait for every MMA this thread issued before TMEM can be released.
-      umma_commit(smem_u32(drain));
+      // Every MMA issued by this thread is complete before TMEM is released.
+      umma_commit_pair(smem_u32(drain), 0x1);
       drain_phase(smem_u32(drain), 0, wc, SITE_DRAIN_MMA);
     }
     __syncwarp();
@@ -287,8 +286,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;  // TMEM lanes [32*quarter, +32) belong to this warp
     const int r = quarter * 32 + lane;
-    Sched sch;
-    sch.init(sa, blockIdx.x, gridDim.x);
+    PairSched sch;
+    sch.init(sa, cluster, nclusters);
     Work w;
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -300,11 +299,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (!ok) break;
       tc_fence_after();
+      w.m0 = w.mt * PM + (int)rank * CM;
+      w.n0 = w.nt * BN;
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
       Epi::tile(ep, st, w, taddr, r, &tmC, quarter, lane);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
@@ -313,8 +314,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();  // neither CTA releases TMEM or exits while the pair still uses it
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+  if (warp == 1) tmem_dealloc_pair(tmem_base, TMEM_COLS);
 }
 
 }  // namespace fckl

@@ -45,16 +45,19 @@ __global__ void __launch_bounds__(1024) k_count_valid(const uint8_t* __restrict_
 }
 
 // Teacher side of one chunk, one warp per row: p = softmax(topk_logit / T)
-// over the K cached logits, sum_k p_k log p_k, and the (id, p) pairs sorted by
-// id so that the GEMM epilogues can walk them while sweeping vocab tiles in
-// increasing order.  Ids outside [0, V) are recorded as an error and replaced
-// by INT_MAX, which no vocab column matches.
+// over the K cached logits, sum_k p_k log p_k, the (id, p) pairs sorted by id,
+// and for every vocab tile of 256 columns the position of its first id in the
+// sorted list (tstart, NT + 1 entries per row), so that a GEMM epilogue finds
+// the cached ids of its tile with one load.  Ids outside [0, V) are recorded
+// as an error and replaced by INT_MAX, which no vocab column matches.
 __global__ void __launch_bounds__(ROW_WARPS * 32)
     k_prep_teacher(const int32_t* __restrict__ ids, const float* __restrict__ lg,
-                   const uint8_t* __restrict__ mask, int rows_c, int K, int V, float invT,
-                   int* __restrict__ sid, float* __restrict__ sp, float* __restrict__ zs,
+                   const uint8_t* __restrict__ mask, int rows_c, int K, int V, int NT,
+                   float invT, int* __restrict__ sid, float* __restrict__ sp,
+                   float* __restrict__ zs, uint16_t* __restrict__ tstart,
                    float* __restrict__ plogp, DeviceCtl* ctl) {
   __shared__ int s_ids[ROW_WARPS][K_MAX];
+  __shared__ int s_sorted[ROW_WARPS][K_MAX];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * ROW_WARPS + warp;
   if (row >= rows_c) return;  // warp-uniform
@@ -117,35 +120,41 @@ __global__ void __launch_bounds__(ROW_WARPS * 32)
       sid[(size_t)row * K + rk] = id[i];
       sp[(size_t)row * K + rk] = p[i];
       zs[(size_t)row * K + rk] = 0.f;
+      s_sorted[warp][rk] = id[i];
     }
+  }
+  __syncwarp();
+  for (int vt = lane; vt <= NT; vt += 32) {  // lower bound of vt * 256 in the sorted ids
+    const long long key = (long long)vt * BN;
+    int lo = 0, hi = K;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if ((long long)s_sorted[warp][mid] < key) lo = mid + 1; else hi = mid;
+    }
+    tstart[(size_t)row * (NT + 1) + vt] = (uint16_t)lo;
   }
   if (lane == 0) plogp[row] = pl;
 }
 
-// Merge the per-segment (max, sum) partials of each row into its log-sum-exp
-// (log2 domain, kept for the backward epilogue) and form the row loss
-//   l_r = sum_k p_k log p_k - sum_k p_k (z_k / T - LSE_r),   0 for masked rows.
+// Merge the per-vocab-tile (max, sum) partials of each row into its
+// log-sum-exp (log2 domain, kept for the backward epilogue) and form the row
+// loss  l_r = sum_k p_k log p_k - sum_k p_k (z_k / T - LSE_r),  0 for masked rows.
 __global__ void __launch_bounds__(ROW_WARPS * 32)
-    k_merge_loss(const float2* __restrict__ partials, int Smax, int NT, long long total, int G,
-                 int rows_c, int K, float invT, const float* __restrict__ zs,
-                 const float* __restrict__ sp, const float* __restrict__ plogp,
-                 const uint8_t* __restrict__ mask, float* __restrict__ lse2_out,
-                 float* __restrict__ row_loss) {
+    k_merge_loss(const float2* __restrict__ partials, int NT, int rows_c, int K, float invT,
+                 const float* __restrict__ zs, const float* __restrict__ sp,
+                 const float* __restrict__ plogp, const uint8_t* __restrict__ mask,
+                 float* __restrict__ lse2_out, float* __restrict__ row_loss) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * ROW_WARPS + warp;
   if (row >= rows_c) return;
-  const int rb = row / BM, r = row - rb * BM;
-  const long long x0 = (long long)rb * NT;
-  const int first = (int)lin_owner(x0, total, G);
-  const int nsplit = (int)lin_owner(x0 + NT - 1, total, G) - first + 1;
-  const float2* pr = partials + (size_t)rb * Smax * BM + r;
+  const float2* pr = partials + (size_t)row * NT;
   float M = -INFINITY;
-  for (int s = lane; s < nsplit; s += 32) M = fmaxf(M, pr[(size_t)s * BM].x);
+  for (int t = lane; t < NT; t += 32) M = fmaxf(M, pr[t].x);
   M = warp_max(M);
   float S = 0.f;
-  for (int s = lane; s < nsplit; s += 32) {
-    const float2 q = pr[(size_t)s * BM];
-    S += q.y * exp2f(q.x - M);
+  for (int t = lane; t < NT; t += 32) {
+    const float2 q = pr[t];
+    if (q.x > -INFINITY) S += q.y * exp2f(q.x - M);
   }
   S = warp_sum(S);
   const float L2 = M + log2f(S);

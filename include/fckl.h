@@ -129,13 +129,18 @@ fckl_status fckl_check(void* workspace, void* stream);
 const char* fckl_status_string(fckl_status status);
 
 /* Optional per-kernel timing for measurement tools.  Between
- * fckl_profile_begin() and fckl_profile_end(), every kernel the library
- * launches is bracketed by two CUDA events recorded on the call's stream
- * (events are created on first use and reused; no device memory is
- * allocated).  fckl_profile_end() synchronises those events, stops recording
- * and writes up to `max_stats` per-kernel summaries (one per kernel kind, in
- * first-launch order); it returns how many kinds were seen, or -1 on a CUDA
- * error.  Recording is process-wide and not thread-safe. */
+ * fckl_profile_begin(mask) and fckl_profile_end(), every kernel the library
+ * launches whose kind is selected by `mask` (bit i = kind i of the list below;
+ * 0 selects every kind) is bracketed by two CUDA events recorded on the
+ * call's stream (events are created on first use and reused; no device
+ * memory is allocated).  Event records between kernels cost time, so select
+ * only the kinds you need while timing a whole call.  fckl_profile_end()
+ * synchronises those events, stops recording and writes up to `max_stats`
+ * per-kernel summaries (one per kind, in first-launch order); it returns how
+ * many kinds were seen, or -1 on a CUDA error.  Recording is process-wide and
+ * not thread-safe.
+ * Kinds: 0 count_valid, 1 prep_teacher, 2 fwd_logits_lse, 3 merge_loss,
+ *        4 bwd_dlogits, 5 dH_gemm, 6 dW_gemm, 7 finalize. */
 typedef struct {
   char name[32];     /* kernel kind, e.g. "fwd_logits_lse" */
   int64_t launches;  /* launches recorded */
@@ -145,7 +150,7 @@ typedef struct {
                         reads + writes of operands and outputs) */
 } fckl_kernel_stat;
 
-void fckl_profile_begin(void);
+void fckl_profile_begin(uint32_t kind_mask);
 int fckl_profile_end(fckl_kernel_stat* stats, int max_stats);
 
 #ifdef __cplusplus
