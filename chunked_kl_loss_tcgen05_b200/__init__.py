@@ -20,6 +20,7 @@ __all__ = [
     "FCKL_K_MAX", "FcklProblem", "FcklError", "load", "lib_path", "exported_symbols",
     "fckl_workspace_bytes", "fckl_resolved_chunk", "fckl_fwd", "fckl_fwd_bwd", "fckl_check",
     "fckl_status_string", "FcklKernelStat", "fckl_profile_begin", "fckl_profile_end",
+    "fckl_fwd_noalloc",
 ]
 
 FCKL_OK = 0
@@ -36,7 +37,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
 
 exported_symbols = ("fckl_workspace_bytes", "fckl_resolved_chunk", "fckl_fwd", "fckl_fwd_bwd",
-                    "fckl_check", "fckl_status_string", "fckl_profile_begin", "fckl_profile_end")
+                    "fckl_check", "fckl_status_string", "fckl_profile_begin", "fckl_profile_end",
+                    "fckl_fwd_noalloc")
 
 
 class FcklProblem(ctypes.Structure):
@@ -89,6 +91,8 @@ def load() -> ctypes.CDLL:
     lib.fckl_check.restype = ctypes.c_int
     lib.fckl_status_string.argtypes = [ctypes.c_int]
     lib.fckl_status_string.restype = ctypes.c_char_p
+    lib.fckl_fwd_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.fckl_fwd_noalloc.restype = ctypes.c_int
     lib.fckl_profile_begin.argtypes = [ctypes.c_uint32]
     lib.fckl_profile_begin.restype = None
     lib.fckl_profile_end.argtypes = [ctypes.POINTER(FcklKernelStat), ctypes.c_int]
@@ -125,6 +129,15 @@ def fckl_fwd_bwd(prob, hidden, W, topk_idx, topk_logit, row_mask, loss, row_loss
                                    _ptr(topk_logit), _ptr(row_mask), _ptr(loss),
                                    _ptr(row_loss), _ptr(dH), _ptr(dW), _ptr(workspace),
                                    ctypes.c_size_t(int(workspace_bytes)), _ptr(stream)))
+
+
+def fckl_fwd_noalloc(prob, hidden, W, topk_idx, topk_logit, row_mask, loss, row_loss,
+                     device_status, stream) -> int:
+    """Forward loss with the library's own static scratch (no workspace, no
+    allocation).  Array arguments are device addresses (ints) or None."""
+    return int(load().fckl_fwd_noalloc(ctypes.byref(prob), _ptr(hidden), _ptr(W), _ptr(topk_idx),
+                                       _ptr(topk_logit), _ptr(row_mask), _ptr(loss),
+                                       _ptr(row_loss), _ptr(device_status), _ptr(stream)))
 
 
 def fckl_check(workspace, stream) -> int:

@@ -57,7 +57,7 @@ long long resolve_chunk(const fckl_problem* p) {
   return std::min<long long>(C, p->N);
 }
 
-Layout make_layout(const fckl_problem* p) {
+Layout make_layout(const fckl_problem* p, bool with_dlogits = true) {
   Layout L{};
   L.N = p->N; L.H = p->H; L.V = p->V; L.K = p->K;
   L.Vp = (long long)align_up((size_t)p->V, 8);
@@ -74,7 +74,7 @@ Layout make_layout(const fckl_problem* p) {
   L.off_plogp = take((size_t)L.C * 4);
   L.off_lse2 = take((size_t)L.C * 4);
   L.off_part = take((size_t)L.C * L.NT * sizeof(float2));
-  L.off_dlog = take((size_t)L.C * L.Vp * 2);
+  L.off_dlog = take(with_dlogits ? (size_t)L.C * L.Vp * 2 : 0);
   L.total = off;
   return L;
 }
@@ -230,7 +230,7 @@ inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_
 fckl_status run(bool bwd, const fckl_problem* prob, const void* hidden, const void* W,
                 const int32_t* topk_idx, const float* topk_logit, const uint8_t* row_mask,
                 float* loss, float* row_loss, float* dH, float* dW, void* workspace,
-                size_t ws_bytes, void* stream_ptr) {
+                size_t ws_bytes, void* stream_ptr, bool fwd_only_layout = false) {
   if (!valid_problem(prob)) return FCKL_ERR_INVALID_ARG;
   if (!hidden || !W || !topk_idx || !topk_logit || !loss) return FCKL_ERR_INVALID_ARG;
   if (bwd && (!dH || !dW)) return FCKL_ERR_INVALID_ARG;
@@ -239,7 +239,7 @@ fckl_status run(bool bwd, const fckl_problem* prob, const void* hidden, const vo
       (bwd && (!aligned(dH, 16) || !aligned(dW, 16))))
     return FCKL_ERR_INVALID_ARG;
   if (!supported_problem(prob)) return FCKL_ERR_UNSUPPORTED;
-  const Layout L = make_layout(prob);
+  const Layout L = make_layout(prob, !(fwd_only_layout && !bwd));
   if (workspace == nullptr || !aligned(workspace, kAlign) || ws_bytes < L.total)
     return FCKL_ERR_WORKSPACE;
   const DeviceInfo* dev = device_info();
@@ -371,9 +371,75 @@ fckl_status run(bool bwd, const fckl_problem* prob, const void* hidden, const vo
   return FCKL_OK;
 }
 
+// ---------------------------------------------------------------- no-alloc forward
+// Library-owned scratch for fckl_fwd_noalloc.  Every GPU that loads the
+// library keeps this array resident until the process exits.
+constexpr size_t kStaticScratchBytes = 32ull << 20;
+__device__ __align__(256) uint8_t g_fwd_scratch[kStaticScratchBytes];
+
+struct StaticScratch {
+  bool ready = false;
+  void* ptr = nullptr;
+};
+StaticScratch g_scratch[kMaxDevices];
+std::mutex g_scratch_mu;
+
+// Device address of g_fwd_scratch on the current device.  In host code the
+// symbol is only a host-side stand-in, so the address is looked up once per
+// device with that device current.
+void* static_scratch() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  StaticScratch& s = g_scratch[dev];
+  if (!s.ready) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_fwd_scratch) != cudaSuccess || p == nullptr) return nullptr;
+    s.ptr = p;
+    s.ready = true;
+  }
+  return s.ptr;
+}
+
+// Device-side error bits of the control block -> fckl_status, for callers
+// that have no workspace to hand to fckl_check().
+__global__ void k_export_status(const DeviceCtl* ctl, int32_t* status_out) {
+  const uint32_t e = ctl->err;
+  *status_out = (e & kErrTimeout)     ? (int32_t)FCKL_ERR_TIMEOUT
+                : (e & kErrBadIndex)  ? (int32_t)FCKL_ERR_BAD_INDEX
+                : (e & kErrBadTeacher) ? (int32_t)FCKL_ERR_BAD_TEACHER
+                                       : (int32_t)FCKL_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+fckl_status fckl_fwd_noalloc(const fckl_problem* prob, const void* hidden, const void* W,
+                             const int32_t* topk_idx, const float* topk_logit,
+                             const uint8_t* row_mask, float* loss, float* row_loss,
+                             int32_t* device_status, void* stream) {
+  if (!valid_problem(prob)) return FCKL_ERR_INVALID_ARG;
+  if (!supported_problem(prob)) return FCKL_ERR_UNSUPPORTED;
+  if (device_status && !aligned(device_status, 4)) return FCKL_ERR_INVALID_ARG;
+  fckl_problem q = *prob;
+  long long C = resolve_chunk(prob);
+  for (;;) {  // the largest chunk (or the caller's chunk) whose scratch fits
+    q.chunk = C;
+    if (make_layout(&q, false).total <= kStaticScratchBytes) break;
+    if (prob->chunk != 0 || C <= PM) return FCKL_ERR_WORKSPACE;
+    C = std::max<long long>(PM, C / 2 / PM * PM);
+  }
+  void* scratch = static_scratch();
+  if (scratch == nullptr) return FCKL_ERR_CUDA;
+  const fckl_status st = run(false, &q, hidden, W, topk_idx, topk_logit, row_mask, loss, row_loss,
+                             nullptr, nullptr, scratch, kStaticScratchBytes, stream, true);
+  if (st != FCKL_OK || device_status == nullptr) return st;
+  k_export_status<<<1, 1, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const DeviceCtl*>(scratch), device_status);
+  return cudaGetLastError() == cudaSuccess ? FCKL_OK : FCKL_ERR_CUDA;
+}
+
 
 size_t fckl_workspace_bytes(const fckl_problem* prob) {
   if (!valid_problem(prob) || !supported_problem(prob)) return 0;

@@ -120,6 +120,37 @@ fckl_status fckl_fwd_bwd(const fckl_problem* prob, const void* hidden, const voi
                          float* dH, float* dW,
                          void* workspace, size_t workspace_bytes, void* stream);
 
+/* Forward only (loss and optional row_loss), like fckl_fwd, but without a
+ * workspace argument: the call allocates nothing and takes no memory from the
+ * caller beyond its inputs and outputs.  It is meant for callers that cannot
+ * call cudaMalloc or hand out scratch buffers -- for example code running
+ * inside a host framework whose own allocator owns all device memory and
+ * forbids side allocations, or a plugin whose interface passes only the
+ * tensors it computes on.  (The pages describe no such entry point; it is an
+ * addition of this library.)
+ *   - Scratch lives in a 32 MiB file-scope __device__ array of the library;
+ *     every GPU that loads the library holds it until the process exits.
+ *   - The first call on a device looks up that array's device address with
+ *     the device current (one cudaGetSymbolAddress per device); make that
+ *     first call before any stream capture on the device.
+ *   - The scratch holds N floats of per-row loss plus the per-chunk teacher
+ *     and log-sum-exp buffers.  prob->chunk = 0 picks the largest multiple of
+ *     256 rows (or N) that fits; an explicit chunk that does not fit, or a
+ *     problem for which even 256 rows do not fit, returns FCKL_ERR_WORKSPACE
+ *     before anything is enqueued.
+ *   - All calls share the one array and each call re-initialises what must
+ *     start at zero; calls that can overlap on the GPU (other streams, other
+ *     host threads) race on it and must be serialised by the caller.
+ *   - device_status (device int32, may be NULL) receives, in stream order, the
+ *     device-side status of this call (FCKL_OK, FCKL_ERR_BAD_INDEX,
+ *     FCKL_ERR_BAD_TEACHER or FCKL_ERR_TIMEOUT) -- the role fckl_check() plays
+ *     for the workspace entry points.
+ * Other arguments, layouts and host-side errors are those of fckl_fwd. */
+fckl_status fckl_fwd_noalloc(const fckl_problem* prob, const void* hidden, const void* W,
+                             const int32_t* topk_idx, const float* topk_logit,
+                             const uint8_t* row_mask, float* loss, float* row_loss,
+                             int32_t* device_status, void* stream);
+
 /* Synchronises `stream`, then returns the first device-side error recorded in
  * `workspace` by the last call that used it (FCKL_OK if none), or
  * FCKL_ERR_CUDA if the stream reports a CUDA error. */

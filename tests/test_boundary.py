@@ -123,3 +123,13 @@ def test_no_gpu_fails_loudly():
     f = 1 << 20
     st = fk.fckl_fwd_bwd(p, f, f, f, f, None, f, None, f, f, f, ws, None)
     assert st in (fk.FCKL_ERR_UNSUPPORTED, fk.FCKL_ERR_CUDA)
+
+
+def test_noalloc_rejects_oversized_problem():
+    """The allocation-free forward refuses, before touching the device, a chunk
+    whose scratch would not fit in the library's static array."""
+    prob = FcklProblem(8192, 4096, 1_000_000, 100, 1.0, 4096)  # ~165 MB of forward scratch
+    f = 1 << 20
+    assert fk.fckl_fwd_noalloc(prob, f, f, f, f, None, f, None, None, None) == fk.FCKL_ERR_WORKSPACE
+    bad = FcklProblem(64, 60, 512, 8, 1.0, 0)  # H % 8 != 0
+    assert fk.fckl_fwd_noalloc(bad, f, f, f, f, None, f, None, None, None) == fk.FCKL_ERR_UNSUPPORTED
