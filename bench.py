@@ -57,6 +57,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=0, help="rows in the oracle sample (0 = auto)")
     ap.add_argument("--profile-json", default="")
+    ap.add_argument("--mem-sweep", action="store_true",
+                    help="print peak device memory vs sequence length instead of timing")
     return ap.parse_args()
 
 
@@ -204,8 +206,11 @@ def run_cuda(args):
     torch.cuda.synchronize()
     torch.cuda.reset_peak_memory_stats(dev)
 
+    outs = (torch.empty(1, device=dev), torch.empty(cfg.N, cfg.H, device=dev),
+            torch.empty(cfg.V, cfg.H, device=dev))
+
     def step():
-        return fused_kl_fwd_bwd(*d, T=cfg.T, chunk=cfg.chunk, workspace=ws, check=False)
+        return fused_kl_fwd_bwd(*d, T=cfg.T, chunk=cfg.chunk, workspace=ws, check=False, out=outs)
 
     from chunked_kl_loss_tcgen05_b200 import fckl_check
     for _ in range(args.warmup):
@@ -287,7 +292,7 @@ def run_cuda(args):
 
     e2e = None
     if not args.no_e2e:
-        e2e = measure_e2e(torch, dev, inp, cfg, ws, max(3, min(args.steps, 5)), world)
+        e2e = measure_e2e(torch, dev, inp, cfg, ws, max(3, min(args.steps, 5)), world, outs)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -323,7 +328,7 @@ def run_cuda(args):
     return 0
 
 
-def measure_e2e(torch, dev, inp, cfg, ws, steps, world):
+def measure_e2e(torch, dev, inp, cfg, ws, steps, world, outs):
     """Same metric through the public API from pinned host buffers: every step
     copies that step's inputs host->device and reads the loss back."""
     from chunked_kl_loss_tcgen05_b200.torch_api import fused_kl_from_host
@@ -335,13 +340,13 @@ def measure_e2e(torch, dev, inp, cfg, ws, steps, world):
     bufs = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     for _ in range(2):
-        fused_kl_from_host(bufs, host, T=cfg.T, chunk=cfg.chunk, workspace=ws)
+        fused_kl_from_host(bufs, host, T=cfg.T, chunk=cfg.chunk, workspace=ws, out=outs)
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(steps):
-        fused_kl_from_host(bufs, host, T=cfg.T, chunk=cfg.chunk, workspace=ws)
+        fused_kl_from_host(bufs, host, T=cfg.T, chunk=cfg.chunk, workspace=ws, out=outs)
     e1.record(stream)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
@@ -350,10 +355,47 @@ def measure_e2e(torch, dev, inp, cfg, ws, steps, world):
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": 4, "steps": steps}
 
 
+def run_mem_sweep(args):
+    """Peak device memory of one fused forward+backward call vs sequence length
+    at the 32K toy-projection shape (H=4096, V=128256, K=100, chunk=2048):
+    inputs, outputs and workspace all counted (torch.cuda.max_memory_allocated)."""
+    import torch
+    from chunked_kl_loss_tcgen05_b200.torch_api import fused_kl_fwd_bwd
+    torch.cuda.set_device(0)
+    H, V, K, C = 4096, 128256, 100, 2048
+    pts = []
+    for S in (8192, 16384, 32768, 65536, 131072, 262144):
+        torch.cuda.empty_cache()
+        base = torch.cuda.memory_allocated()
+        g = torch.Generator(device="cuda").manual_seed(S)
+        hidden = torch.randn(S, H, device="cuda", dtype=torch.bfloat16, generator=g)
+        W = (torch.randn(V, H, device="cuda", generator=g) * 0.02).to(torch.bfloat16)
+        ids = torch.randint(0, V, (S, K), device="cuda", dtype=torch.int32, generator=g)
+        lg = torch.randn(S, K, device="cuda", generator=g) * 3
+        torch.cuda.synchronize()
+        torch.cuda.reset_peak_memory_stats()  # inputs stay counted, their fp32 temporaries do not
+        loss, _, dH, dW = fused_kl_fwd_bwd(hidden, W, ids, lg, None, T=1.0, chunk=C)
+        torch.cuda.synchronize()
+        peak = (torch.cuda.max_memory_allocated() - base) / 2**30
+        pts.append((S, peak))
+        del hidden, W, ids, lg, loss, dH, dW
+    xs = np.array([p[0] for p in pts], dtype=np.float64)
+    ys = np.array([p[1] for p in pts], dtype=np.float64)
+    b, a = np.polyfit(xs, ys, 1)
+    r2 = 1 - ((ys - (a + b * xs)) ** 2).sum() / ((ys - ys.mean()) ** 2).sum()
+    line = {"metric": "peak GiB vs seq len (fused fwd+bwd, H=4096 V=128256 K=100 chunk=2048)",
+            "points": [{"S": s, "peak_gib": round(p, 4)} for s, p in pts],
+            "fit": {"intercept_gib": a, "slope_kib_per_row": b * 2**20, "r2": r2}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.mem_sweep:
+        return run_mem_sweep(args)
     return run_cuda(args)
 
 

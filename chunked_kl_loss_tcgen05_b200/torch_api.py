@@ -51,18 +51,27 @@ def _check_inputs(hidden, W, topk_idx, topk_logit, row_mask):
 
 
 def fused_kl_fwd_bwd(hidden, W, topk_idx, topk_logit, row_mask=None, T=1.0, chunk=0,
-                     workspace=None, want_row_loss=False, check=True):
-    """Returns (loss[1], row_loss[N] or None, dH[N,H] fp32, dW[V,H] fp32)."""
+                     workspace=None, want_row_loss=False, check=True, out=None):
+    """Returns (loss[1], row_loss[N] or None, dH[N,H] fp32, dW[V,H] fp32).
+
+    ``out``: optional (loss, dH, dW) tensors to write into instead of allocating."""
     hidden, W = _bits(hidden), _bits(W)
     _check_inputs(hidden, W, topk_idx, topk_logit, row_mask)
     prob = make_problem(hidden, W, topk_idx, T, chunk)
     dev = hidden.device
     if workspace is None:
         workspace = alloc_workspace(prob, dev)
-    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    if out is not None:
+        loss, dH, dW = out
+        if (loss.numel() < 1 or tuple(dH.shape) != (prob.N, prob.H)
+                or tuple(dW.shape) != (prob.V, prob.H) or dH.dtype != torch.float32
+                or dW.dtype != torch.float32 or not dH.is_contiguous() or not dW.is_contiguous()):
+            raise ValueError("out must be (loss[>=1], dH[N,H], dW[V,H]) contiguous float32")
+    else:
+        loss = torch.empty(1, dtype=torch.float32, device=dev)
+        dH = torch.empty(prob.N, prob.H, dtype=torch.float32, device=dev)
+        dW = torch.empty(prob.V, prob.H, dtype=torch.float32, device=dev)
     row_loss = torch.empty(prob.N, dtype=torch.float32, device=dev) if want_row_loss else None
-    dH = torch.empty(prob.N, prob.H, dtype=torch.float32, device=dev)
-    dW = torch.empty(prob.V, prob.H, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev).cuda_stream
     st = fckl_fwd_bwd(prob, hidden.data_ptr(), W.data_ptr(), topk_idx.data_ptr(),
                       topk_logit.data_ptr(), None if row_mask is None else row_mask.data_ptr(),
@@ -103,7 +112,7 @@ def fused_kl_fwd(hidden, W, topk_idx, topk_logit, row_mask=None, T=1.0, chunk=0,
     return loss, row_loss
 
 
-def fused_kl_from_host(dev_bufs: dict, host: dict, T=1.0, chunk=0, workspace=None):
+def fused_kl_from_host(dev_bufs: dict, host: dict, T=1.0, chunk=0, workspace=None, out=None):
     """End-to-end call from pinned host arrays: copies the inputs host->device on
     the current stream, runs fused forward+backward, and reads the loss back.
     ``dev_bufs`` holds preallocated device tensors with the same keys as
@@ -113,7 +122,7 @@ def fused_kl_from_host(dev_bufs: dict, host: dict, T=1.0, chunk=0, workspace=Non
         dev_bufs[k].copy_(h, non_blocking=True)
     loss, _, dH, dW = fused_kl_fwd_bwd(dev_bufs["hidden"], dev_bufs["W"], dev_bufs["topk_idx"],
                                        dev_bufs["topk_logit"], dev_bufs.get("row_mask"), T=T,
-                                       chunk=chunk, workspace=workspace, check=False)
+                                       chunk=chunk, workspace=workspace, check=False, out=out)
     return float(loss.item()), dH, dW
 
 
