@@ -24,11 +24,14 @@ namespace {
 constexpr size_t kAlign = 256;
 constexpr int kMaxDevices = 64;
 
+constexpr long long kDwRows = 2048;  // minimum reduction depth of a dW launch (rows)
+
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
 
 struct Layout {
   long long N, H, V, K, C, Vp, nchunks, NT;
+  long long G;  // chunks per dW group: dlogits of G chunks feed one dW GEMM
   size_t off_rowloss, off_sid, off_sp, off_zs, off_tstart, off_plogp, off_lse2, off_part,
       off_dlog, total;
 };
@@ -63,6 +66,10 @@ Layout make_layout(const fckl_problem* p, bool with_dlogits = true) {
   L.Vp = (long long)align_up((size_t)p->V, 8);
   L.C = resolve_chunk(p);
   L.nchunks = cdiv(L.N, L.C);
+  // The dW GEMM reduces over the rows of its dlogits block, and each launch
+  // reads and writes dW once (fp32, V*H*8 bytes).  Small chunks are grouped
+  // so that one dW launch covers at least kDwRows rows.
+  L.G = std::min<long long>(L.nchunks, std::max<long long>(1, cdiv(kDwRows, L.C)));
   L.NT = cdiv(L.V, BN);
   size_t off = align_up(sizeof(DeviceCtl), kAlign);
   auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, kAlign); return o; };
@@ -74,7 +81,7 @@ Layout make_layout(const fckl_problem* p, bool with_dlogits = true) {
   L.off_plogp = take((size_t)L.C * 4);
   L.off_lse2 = take((size_t)L.C * 4);
   L.off_part = take((size_t)L.C * L.NT * sizeof(float2));
-  L.off_dlog = take(with_dlogits ? (size_t)L.C * L.Vp * 2 : 0);
+  L.off_dlog = take(with_dlogits ? (size_t)L.G * L.C * L.Vp * 2 : 0);
   L.total = off;
   return L;
 }
@@ -211,7 +218,8 @@ struct ProfScope {
 };
 
 // Split-K factor for dH: minimise waves * (k-blocks per unit + fixed cost),
-// with `slots` CTA pairs working at once.
+// with `slots` CTA pairs working at once.  (Capping the k-segment to keep it
+// L2-resident cut DRAM reads but made the kernel slower: more, shorter units.)
 int choose_split(long long tiles, long long KB, int slots) {
   int best = 1;
   double best_cost = 1e300;
@@ -288,6 +296,8 @@ fckl_status run(bool bwd, const fckl_problem* prob, const void* hidden, const vo
     const uint8_t* mask_c = row_mask ? row_mask + row0 : nullptr;
     const void* h_c = static_cast<const uint8_t*>(hidden) + (size_t)row0 * L.H * 2;
     const int row_blocks = (int)cdiv(rows, ROW_WARPS);
+    // This chunk's rows in the group's dlogits block.
+    __nv_bfloat16* dlog_c = dlog + (size_t)(c % L.G) * L.C * L.Vp;
 
     {
       ProfScope ps(K_PREP, st, 0.0, (double)rows * K * 20.0 + rows * (NT + 1) * 2.0);
@@ -322,7 +332,7 @@ fckl_status run(bool bwd, const fckl_problem* prob, const void* hidden, const vo
     // Backward 1: recompute the tiles and form bf16 dlogits = q - p~.
     EpiDlogits::Params pb{rows, V, K, (int)NT, scale2, lse2, sid, tstart, sp, mask_c};
     CUtensorMap mapD_st;
-    if (!make_map(&mapD_st, dlog, L.V, rows, L.Vp * 2, 64, 32)) return FCKL_ERR_CUDA;
+    if (!make_map(&mapD_st, dlog_c, L.V, rows, L.Vp * 2, 64, 32)) return FCKL_ERR_CUDA;
     {
       ProfScope ps(K_BWD, st, gemm_flops, 2.0 * (rows + (double)L.V) * L.H + 2.0 * rows * L.V);
       gemm_pair_kernel<EpiDlogits, false, false>
@@ -334,7 +344,7 @@ fckl_status run(bool bwd, const fckl_problem* prob, const void* hidden, const vo
     if (cudaMemsetAsync(dH + row0 * L.H, 0, (size_t)rows * L.H * 4, st) != cudaSuccess)
       return FCKL_ERR_CUDA;
     CUtensorMap mapD_k, mapD_mn, mapH_mn, mapdH;
-    if (!make_map(&mapD_k, dlog, L.V, rows, L.Vp * 2, BK, CM)) return FCKL_ERR_CUDA;
+    if (!make_map(&mapD_k, dlog_c, L.V, rows, L.Vp * 2, BK, CM)) return FCKL_ERR_CUDA;
     if (!make_map(&mapdH, dH + row0 * L.H, L.H, rows, L.H * 4, 32, 32, true)) return FCKL_ERR_CUDA;
     const long long tiles_h = MT * NTh;
     const int S = choose_split(tiles_h, KBv, pairs);
@@ -348,16 +358,23 @@ fckl_status run(bool bwd, const fckl_problem* prob, const void* hidden, const vo
               mapD_k, mapW_mn, mapdH, ph, sa_h, ca);
     }
 
-    // Backward 3: dW (+)= alpha * dlogits^T h; A = dlogits^T, B = h (both MN-major).
-    if (!make_map(&mapD_mn, dlog, L.V, rows, L.Vp * 2, 64, BK)) return FCKL_ERR_CUDA;
-    if (!make_map(&mapH_mn, h_c, L.H, rows, L.H * 2, 64, BK)) return FCKL_ERR_CUDA;
+    // Backward 3, once per group of G chunks (or at the last chunk):
+    // dW (+)= alpha * dlogits^T h over the group's rows; A = dlogits^T, B = h
+    // (both MN-major).
+    if ((c + 1) % L.G != 0 && c + 1 != L.nchunks) continue;
+    const long long g0 = c / L.G * L.G;  // first chunk of the group
+    const long long grow0 = g0 * L.C;
+    const int grows = (int)(row0 + rows - grow0);
+    const void* h_g = static_cast<const uint8_t*>(hidden) + (size_t)grow0 * L.H * 2;
+    if (!make_map(&mapD_mn, dlog, L.V, grows, L.Vp * 2, 64, BK)) return FCKL_ERR_CUDA;
+    if (!make_map(&mapH_mn, h_g, L.H, grows, L.H * 2, 64, BK)) return FCKL_ERR_CUDA;
     const long long tiles_w = cdiv(L.V, PM) * NTh;
-    SchedArgs sa_w{tiles_w, SCHED_TILES, 0, (int)NTh, (int)cdiv(rows, BK), 1, (int)tiles_w};
-    EpiDW::Params pw{V, H, invT, c > 0 ? 1 : 0, ctl};
+    SchedArgs sa_w{tiles_w, SCHED_TILES, 0, (int)NTh, (int)cdiv(grows, BK), 1, (int)tiles_w};
+    EpiDW::Params pw{V, H, invT, g0 > 0 ? 1 : 0, ctl};
     {
-      ProfScope ps(K_DW, st, gemm_flops,
-                   2.0 * rows * (double)L.V + 2.0 * rows * L.H +
-                       (c > 0 ? 8.0 : 4.0) * (double)L.V * L.H);
+      ProfScope ps(K_DW, st, 2.0 * grows * (double)L.V * (double)L.H,
+                   2.0 * grows * (double)L.V + 2.0 * grows * L.H +
+                       (g0 > 0 ? 8.0 : 4.0) * (double)L.V * L.H);
       gemm_pair_kernel<EpiDW, true, true>
           <<<grid_for(tiles_w), GEMM_THREADS, pair_smem_bytes<EpiDW>(), st>>>(
               mapD_mn, mapH_mn, mapdW, pw, sa_w, ca);
