@@ -20,7 +20,7 @@ __all__ = [
     "FCKL_K_MAX", "FcklProblem", "FcklError", "load", "lib_path", "exported_symbols",
     "fckl_workspace_bytes", "fckl_resolved_chunk", "fckl_fwd", "fckl_fwd_bwd", "fckl_check",
     "fckl_status_string", "FcklKernelStat", "fckl_profile_begin", "fckl_profile_end",
-    "fckl_fwd_noalloc",
+    "fckl_fwd_noalloc", "fckl_student_entropy", "fckl_select_top_rows", "fckl_fwd_bwd_rows",
 ]
 
 FCKL_OK = 0
@@ -38,7 +38,8 @@ _LIB = None
 
 exported_symbols = ("fckl_workspace_bytes", "fckl_resolved_chunk", "fckl_fwd", "fckl_fwd_bwd",
                     "fckl_check", "fckl_status_string", "fckl_profile_begin", "fckl_profile_end",
-                    "fckl_fwd_noalloc")
+                    "fckl_fwd_noalloc", "fckl_student_entropy", "fckl_select_top_rows",
+                    "fckl_fwd_bwd_rows")
 
 
 class FcklProblem(ctypes.Structure):
@@ -91,6 +92,13 @@ def load() -> ctypes.CDLL:
     lib.fckl_check.restype = ctypes.c_int
     lib.fckl_status_string.argtypes = [ctypes.c_int]
     lib.fckl_status_string.restype = ctypes.c_char_p
+    lib.fckl_student_entropy.argtypes = [P, vp, vp, vp, vp, vp, sz, vp]
+    lib.fckl_student_entropy.restype = ctypes.c_int
+    lib.fckl_select_top_rows.argtypes = [vp, vp, ctypes.c_int64, ctypes.c_int64, vp, vp, vp]
+    lib.fckl_select_top_rows.restype = ctypes.c_int
+    lib.fckl_fwd_bwd_rows.argtypes = [P, vp, vp, vp, vp, vp, ctypes.c_int64, vp, vp, vp, vp, vp,
+                                      sz, vp]
+    lib.fckl_fwd_bwd_rows.restype = ctypes.c_int
     lib.fckl_fwd_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.fckl_fwd_noalloc.restype = ctypes.c_int
     lib.fckl_profile_begin.argtypes = [ctypes.c_uint32]
@@ -140,6 +148,28 @@ def fckl_fwd_noalloc(prob, hidden, W, topk_idx, topk_logit, row_mask, loss, row_
                                        _ptr(row_loss), _ptr(device_status), _ptr(stream)))
 
 
+def fckl_student_entropy(prob, hidden, W, row_mask, row_entropy, workspace, workspace_bytes,
+                         stream) -> int:
+    return int(load().fckl_student_entropy(ctypes.byref(prob), _ptr(hidden), _ptr(W),
+                                           _ptr(row_mask), _ptr(row_entropy), _ptr(workspace),
+                                           ctypes.c_size_t(int(workspace_bytes)), _ptr(stream)))
+
+
+def fckl_select_top_rows(score, row_mask, N, n_select, rows_out, count_out, stream) -> int:
+    return int(load().fckl_select_top_rows(_ptr(score), _ptr(row_mask), ctypes.c_int64(int(N)),
+                                           ctypes.c_int64(int(n_select)), _ptr(rows_out),
+                                           _ptr(count_out), _ptr(stream)))
+
+
+def fckl_fwd_bwd_rows(prob, hidden, W, topk_idx, topk_logit, rows, n_rows, loss, row_loss, dH, dW,
+                      workspace, workspace_bytes, stream) -> int:
+    return int(load().fckl_fwd_bwd_rows(ctypes.byref(prob), _ptr(hidden), _ptr(W), _ptr(topk_idx),
+                                        _ptr(topk_logit), _ptr(rows), ctypes.c_int64(int(n_rows)),
+                                        _ptr(loss), _ptr(row_loss), _ptr(dH), _ptr(dW),
+                                        _ptr(workspace), ctypes.c_size_t(int(workspace_bytes)),
+                                        _ptr(stream)))
+
+
 def fckl_check(workspace, stream) -> int:
     return int(load().fckl_check(_ptr(workspace), _ptr(stream)))
 
@@ -149,7 +179,8 @@ def fckl_status_string(status: int) -> str:
 
 
 KERNEL_KINDS = ("count_valid", "prep_teacher", "fwd_logits_lse", "merge_loss", "bwd_dlogits",
-                "dH_gemm", "dW_gemm", "finalize")
+                "dH_gemm", "dW_gemm", "finalize", "entropy_gemm", "merge_entropy", "gather_rows",
+                "scatter_rows", "select_rows")
 
 
 def fckl_profile_begin(kinds=None) -> None:

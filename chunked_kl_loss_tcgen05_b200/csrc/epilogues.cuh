@@ -37,7 +37,11 @@ __device__ __forceinline__ void tmem_ld32_conv(uint32_t taddr, float (&v)[32]) {
   tmem_ld32(taddr, v);
 }
 
-struct EpiLse {
+// kGather: gather z at the cached teacher ids (loss path).
+// kEntropy: also accumulate sum 2^(a - max) * a per tile, so that the merge can
+// form the student entropy H(q) = ln2 * (LSE2 - U / S) (student-entropy pass).
+template <bool kGather, bool kEntropy>
+struct EpiLseT {
   static constexpr uint32_t kSmemBytes = 0;
   static constexpr bool kUsesMapC = false;
   struct Params {
@@ -48,6 +52,7 @@ struct EpiLse {
     const uint16_t* tstart;   // [rows_c, NT + 1] first sorted position of each vocab tile
     float* zs;                // [rows_c, K] gathered z, same order as sid
     float2* partials;         // [rows_c, NT] (max, sum) in the log2 domain
+    float* upart;             // [rows_c, NT] sum 2^(a - max) * a (kEntropy only)
   };
   struct State {};
   static __device__ void init(const Params&, State&, uint8_t*, int) {}
@@ -57,28 +62,31 @@ struct EpiLse {
     const bool rv = row < p.rows_c;
     const int* rid = p.sid + (size_t)(rv ? row : 0) * p.K;
     int cur = 0, nid = INT_MAX;
-    if (rv) {
+    if (kGather && rv) {
       cur = __ldg(p.tstart + (size_t)row * (p.NT + 1) + w.nt);
       nid = cur < p.K ? __ldg(rid + cur) : INT_MAX;
     }
-    float m = -INFINITY, s = 0.f;
+    float m = -INFINITY, s = 0.f, u = 0.f;
 #pragma unroll 1
     for (int c = 0; c < BN / 32; ++c) {
       float v[32];
       tmem_ld32_conv(taddr + (uint32_t)(c * 32), v);
       if (!rv) continue;
       const int base = w.n0 + c * 32;
-      while (nid < base + 32) {  // gather z at cached ids in this 32-column slice
-        const int j = nid - base;
-        float z = 0.f;
+      if (kGather) {
+        while (nid < base + 32) {  // gather z at cached ids in this 32-column slice
+          const int j = nid - base;
+          float z = 0.f;
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) z = (jj == j) ? v[jj] : z;
-        p.zs[(size_t)row * p.K + cur] = z;
-        ++cur;
-        nid = cur < p.K ? __ldg(rid + cur) : INT_MAX;
+          for (int jj = 0; jj < 32; ++jj) z = (jj == j) ? v[jj] : z;
+          p.zs[(size_t)row * p.K + cur] = z;
+          ++cur;
+          nid = cur < p.K ? __ldg(rid + cur) : INT_MAX;
+        }
       }
       float cm = -INFINITY;
-      if (base + 32 <= p.V) {
+      const bool full = base + 32 <= p.V;
+      if (full) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) { v[j] *= p.scale2; cm = fmaxf(cm, v[j]); }
       } else {
@@ -90,16 +98,27 @@ struct EpiLse {
       }
       if (cm == -INFINITY) continue;
       const float nm = fmaxf(m, cm);
-      float acc = 0.f;
+      const float rescale = exp2f(m - nm);
+      float acc = 0.f, uacc = 0.f;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) acc += exp2f(v[j] - nm);
-      s = s * exp2f(m - nm) + acc;
+      for (int j = 0; j < 32; ++j) {
+        const float e = exp2f(v[j] - nm);
+        acc += e;
+        if (kEntropy) uacc += (full || e > 0.f) ? e * v[j] : 0.f;
+      }
+      s = s * rescale + acc;
+      if (kEntropy) u = u * rescale + uacc;
       m = nm;
     }
-    if (rv) p.partials[(size_t)row * p.NT + w.nt] = make_float2(m, s);
+    if (rv) {
+      p.partials[(size_t)row * p.NT + w.nt] = make_float2(m, s);
+      if (kEntropy) p.upart[(size_t)row * p.NT + w.nt] = u;
+    }
   }
   static __device__ void finish(const Params&, State&, int) {}
 };
+using EpiLse = EpiLseT<true, false>;
+using EpiEntropy = EpiLseT<false, true>;
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);

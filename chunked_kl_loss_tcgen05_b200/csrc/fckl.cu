@@ -33,6 +33,7 @@ struct Layout {
   long long N, H, V, K, C, Vp, nchunks, NT;
   long long G;  // chunks per dW group: dlogits of G chunks feed one dW GEMM
   size_t off_rowloss, off_sid, off_sp, off_zs, off_tstart, off_plogp, off_lse2, off_part,
+      off_upart, off_hstage, off_idstage, off_lgstage, off_mstage, off_dhstage, off_rlstage,
       off_dlog, total;
 };
 
@@ -60,7 +61,9 @@ long long resolve_chunk(const fckl_problem* p) {
   return std::min<long long>(C, p->N);
 }
 
-Layout make_layout(const fckl_problem* p, bool with_dlogits = true) {
+// full = false: the forward-loss-only layout (no dlogits, no entropy or
+// row-list buffers), used by the allocation-free entry point.
+Layout make_layout(const fckl_problem* p, bool full = true) {
   Layout L{};
   L.N = p->N; L.H = p->H; L.V = p->V; L.K = p->K;
   L.Vp = (long long)align_up((size_t)p->V, 8);
@@ -73,15 +76,24 @@ Layout make_layout(const fckl_problem* p, bool with_dlogits = true) {
   L.NT = cdiv(L.V, BN);
   size_t off = align_up(sizeof(DeviceCtl), kAlign);
   auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, kAlign); return o; };
+  const size_t C = (size_t)L.C;
   L.off_rowloss = take((size_t)L.N * 4);
-  L.off_sid = take((size_t)L.C * L.K * 4);
-  L.off_sp = take((size_t)L.C * L.K * 4);
-  L.off_zs = take((size_t)L.C * L.K * 4);
-  L.off_tstart = take((size_t)L.C * (L.NT + 1) * 2);
-  L.off_plogp = take((size_t)L.C * 4);
-  L.off_lse2 = take((size_t)L.C * 4);
-  L.off_part = take((size_t)L.C * L.NT * sizeof(float2));
-  L.off_dlog = take(with_dlogits ? (size_t)L.G * L.C * L.Vp * 2 : 0);
+  L.off_sid = take(C * L.K * 4);
+  L.off_sp = take(C * L.K * 4);
+  L.off_zs = take(C * L.K * 4);
+  L.off_tstart = take(C * (L.NT + 1) * 2);
+  L.off_plogp = take(C * 4);
+  L.off_lse2 = take(C * 4);
+  L.off_part = take(C * L.NT * sizeof(float2));
+  L.off_upart = take(full ? C * L.NT * 4 : 0);
+  // Row-list calls gather their rows into these staging buffers.
+  L.off_hstage = take(full ? (size_t)L.G * C * L.H * 2 : 0);
+  L.off_idstage = take(full ? C * L.K * 4 : 0);
+  L.off_lgstage = take(full ? C * L.K * 4 : 0);
+  L.off_mstage = take(full ? C : 0);
+  L.off_dhstage = take(full ? C * L.H * 4 : 0);
+  L.off_rlstage = take(full ? C * 4 : 0);
+  L.off_dlog = take(full ? (size_t)L.G * C * L.Vp * 2 : 0);
   L.total = off;
   return L;
 }
@@ -153,7 +165,8 @@ const DeviceInfo* device_info() {
     d.ok = major == 10 && minor == 0 && d.sms > 0;
     if (d.ok) {
       d.ok = set_smem_attr<EpiLse, false, false>() && set_smem_attr<EpiDlogits, false, false>() &&
-             set_smem_attr<EpiDH, false, true>() && set_smem_attr<EpiDW, true, true>();
+             set_smem_attr<EpiDH, false, true>() && set_smem_attr<EpiDW, true, true>() &&
+             set_smem_attr<EpiEntropy, false, false>();
     }
   }
   return &d;
@@ -173,10 +186,14 @@ int debug_skip_commit() {
 }
 
 // ---------------------------------------------------------------- profiling
-enum Kind { K_COUNT, K_PREP, K_FWD, K_MERGE, K_BWD, K_DH, K_DW, K_FINAL, K_NKINDS };
-const char* const kKindName[K_NKINDS] = {"count_valid", "prep_teacher", "fwd_logits_lse",
-                                         "merge_loss", "bwd_dlogits", "dH_gemm", "dW_gemm",
-                                         "finalize"};
+enum Kind {
+  K_COUNT, K_PREP, K_FWD, K_MERGE, K_BWD, K_DH, K_DW, K_FINAL, K_ENT, K_ENT_MERGE, K_GATHER,
+  K_SCATTER, K_SELECT, K_NKINDS
+};
+const char* const kKindName[K_NKINDS] = {
+    "count_valid", "prep_teacher", "fwd_logits_lse", "merge_loss", "bwd_dlogits",
+    "dH_gemm",     "dW_gemm",      "finalize",       "entropy_gemm", "merge_entropy",
+    "gather_rows", "scatter_rows", "select_rows"};
 struct ProfRec {
   int kind;
   cudaEvent_t a, b;
@@ -235,29 +252,63 @@ int choose_split(long long tiles, long long KB, int slots) {
 
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-fckl_status run(bool bwd, const fckl_problem* prob, const void* hidden, const void* W,
-                const int32_t* topk_idx, const float* topk_logit, const uint8_t* row_mask,
-                float* loss, float* row_loss, float* dH, float* dW, void* workspace,
-                size_t ws_bytes, void* stream_ptr, bool fwd_only_layout = false) {
+enum class Mode { kFwd, kFwdBwd, kEntropy };
+
+// Everything one library call asks for.  rows == nullptr: the rows are
+// 0..N-1 (row_mask optional); otherwise the call covers the n_rows listed
+// rows (negative entries are skipped) and gathers them chunk by chunk.
+struct Request {
+  Mode mode = Mode::kFwd;
+  const fckl_problem* prob = nullptr;
+  const void* hidden = nullptr;
+  const void* W = nullptr;
+  const int32_t* topk_idx = nullptr;
+  const float* topk_logit = nullptr;
+  const uint8_t* row_mask = nullptr;
+  const int32_t* rows = nullptr;
+  long long n_rows = 0;
+  float* loss = nullptr;
+  float* row_loss = nullptr;
+  float* dH = nullptr;
+  float* dW = nullptr;
+  float* entropy = nullptr;
+  void* workspace = nullptr;
+  size_t ws_bytes = 0;
+  void* stream = nullptr;
+  bool full_layout = true;
+};
+
+fckl_status run(const Request& q) {
+  const fckl_problem* prob = q.prob;
+  const bool bwd = q.mode == Mode::kFwdBwd;
+  const bool ent = q.mode == Mode::kEntropy;
+  const bool list = q.rows != nullptr;
   if (!valid_problem(prob)) return FCKL_ERR_INVALID_ARG;
-  if (!hidden || !W || !topk_idx || !topk_logit || !loss) return FCKL_ERR_INVALID_ARG;
-  if (bwd && (!dH || !dW)) return FCKL_ERR_INVALID_ARG;
-  if (!aligned(hidden, 16) || !aligned(W, 16) || !aligned(topk_idx, 4) ||
-      !aligned(topk_logit, 4) || !aligned(loss, 4) || (row_loss && !aligned(row_loss, 4)) ||
-      (bwd && (!aligned(dH, 16) || !aligned(dW, 16))))
+  if (!q.hidden || !q.W || !aligned(q.hidden, 16) || !aligned(q.W, 16)) return FCKL_ERR_INVALID_ARG;
+  if (ent) {
+    if (!q.entropy || !aligned(q.entropy, 4)) return FCKL_ERR_INVALID_ARG;
+  } else {
+    if (!q.topk_idx || !q.topk_logit || !q.loss) return FCKL_ERR_INVALID_ARG;
+    if (!aligned(q.topk_idx, 4) || !aligned(q.topk_logit, 4) || !aligned(q.loss, 4) ||
+        (q.row_loss && !aligned(q.row_loss, 4)))
+      return FCKL_ERR_INVALID_ARG;
+  }
+  if (bwd && (!q.dH || !q.dW || !aligned(q.dH, 16) || !aligned(q.dW, 16)))
+    return FCKL_ERR_INVALID_ARG;
+  if (list && (q.n_rows < 1 || q.n_rows > INT32_MAX || !aligned(q.rows, 4)))
     return FCKL_ERR_INVALID_ARG;
   if (!supported_problem(prob)) return FCKL_ERR_UNSUPPORTED;
-  const Layout L = make_layout(prob, !(fwd_only_layout && !bwd));
-  if (workspace == nullptr || !aligned(workspace, kAlign) || ws_bytes < L.total)
+  const Layout L = make_layout(prob, q.full_layout);
+  if (q.workspace == nullptr || !aligned(q.workspace, kAlign) || q.ws_bytes < L.total)
     return FCKL_ERR_WORKSPACE;
   const DeviceInfo* dev = device_info();
   if (dev == nullptr || !dev->ok) return FCKL_ERR_UNSUPPORTED;
   if (get_encode_fn() == nullptr) return FCKL_ERR_CUDA;
 
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream_ptr);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(q.stream);
+  uint8_t* ws = static_cast<uint8_t*>(q.workspace);
   DeviceCtl* ctl = reinterpret_cast<DeviceCtl*>(ws);
-  float* rl = row_loss ? row_loss : reinterpret_cast<float*>(ws + L.off_rowloss);
+  float* rl = q.row_loss ? q.row_loss : reinterpret_cast<float*>(ws + L.off_rowloss);
   int* sid = reinterpret_cast<int*>(ws + L.off_sid);
   float* sp = reinterpret_cast<float*>(ws + L.off_sp);
   float* zs = reinterpret_cast<float*>(ws + L.off_zs);
@@ -265,6 +316,13 @@ fckl_status run(bool bwd, const fckl_problem* prob, const void* hidden, const vo
   float* plogp = reinterpret_cast<float*>(ws + L.off_plogp);
   float* lse2 = reinterpret_cast<float*>(ws + L.off_lse2);
   float2* part = reinterpret_cast<float2*>(ws + L.off_part);
+  float* upart = reinterpret_cast<float*>(ws + L.off_upart);
+  __nv_bfloat16* hstage = reinterpret_cast<__nv_bfloat16*>(ws + L.off_hstage);
+  int32_t* idstage = reinterpret_cast<int32_t*>(ws + L.off_idstage);
+  float* lgstage = reinterpret_cast<float*>(ws + L.off_lgstage);
+  uint8_t* mstage = ws + L.off_mstage;
+  float* dhstage = reinterpret_cast<float*>(ws + L.off_dhstage);
+  float* rlstage = reinterpret_cast<float*>(ws + L.off_rlstage);
   __nv_bfloat16* dlog = reinterpret_cast<__nv_bfloat16*>(ws + L.off_dlog);
 
   const int H = (int)L.H, V = (int)L.V, K = (int)L.K;
@@ -273,49 +331,100 @@ fckl_status run(bool bwd, const fckl_problem* prob, const void* hidden, const vo
   CtlArgs ca{ctl, wait_timeout_ns(), debug_skip_commit()};
 
   if (cudaMemsetAsync(ctl, 0, sizeof(DeviceCtl), st) != cudaSuccess) return FCKL_ERR_CUDA;
-  {
-    ProfScope ps(K_COUNT, st, 0.0, row_mask ? (double)L.N : 0.0);
-    k_count_valid<<<1, 1024, 0, st>>>(row_mask, L.N, ctl);
+  if (!ent) {
+    ProfScope ps(K_COUNT, st, 0.0, list ? q.n_rows * 4.0 : (q.row_mask ? (double)L.N : 0.0));
+    if (list)
+      k_count_list<<<1, 1024, 0, st>>>(q.rows, q.n_rows, L.N, ctl);
+    else
+      k_count_valid<<<1, 1024, 0, st>>>(q.row_mask, L.N, ctl);
+  }
+  if (list) {  // rows that are not listed get zero row loss and zero dH
+    if (cudaMemsetAsync(rl, 0, (size_t)L.N * 4, st) != cudaSuccess) return FCKL_ERR_CUDA;
+    if (bwd && cudaMemsetAsync(q.dH, 0, (size_t)L.N * L.H * 4, st) != cudaSuccess)
+      return FCKL_ERR_CUDA;
   }
 
   CUtensorMap mapW_k, mapW_mn, mapdW;
-  if (!make_map(&mapW_k, W, L.H, L.V, L.H * 2, BK, BN / 2)) return FCKL_ERR_CUDA;
-  if (bwd && !make_map(&mapW_mn, W, L.H, L.V, L.H * 2, 64, BK)) return FCKL_ERR_CUDA;
-  if (bwd && !make_map(&mapdW, dW, L.H, L.V, L.H * 4, 32, 32, true)) return FCKL_ERR_CUDA;
+  if (!make_map(&mapW_k, q.W, L.H, L.V, L.H * 2, BK, BN / 2)) return FCKL_ERR_CUDA;
+  if (bwd && !make_map(&mapW_mn, q.W, L.H, L.V, L.H * 2, 64, BK)) return FCKL_ERR_CUDA;
+  if (bwd && !make_map(&mapdW, q.dW, L.H, L.V, L.H * 4, 32, 32, true)) return FCKL_ERR_CUDA;
 
   const int pairs = std::max(1, dev->sms / 2);  // CTA pairs that run at once
   const long long NT = L.NT;
   const long long KBh = cdiv(L.H, BK);
   const long long NTh = cdiv(L.H, BN);
   const long long KBv = cdiv(L.V, BK);
+  const long long R = list ? q.n_rows : L.N;  // rows (or list entries) to process
+  const long long nchunks = cdiv(R, L.C);
+  const long long G = std::min<long long>(nchunks, L.G);
   auto grid_for = [&](long long units) { return (int)(2 * std::min<long long>(pairs, units)); };
-  for (long long c = 0; c < L.nchunks; ++c) {
+  for (long long c = 0; c < nchunks; ++c) {
     const long long row0 = c * L.C;
-    const int rows = (int)std::min(L.C, L.N - row0);
+    const int rows = (int)std::min(L.C, R - row0);
     const long long MT = cdiv(rows, PM);
-    const uint8_t* mask_c = row_mask ? row_mask + row0 : nullptr;
-    const void* h_c = static_cast<const uint8_t*>(hidden) + (size_t)row0 * L.H * 2;
     const int row_blocks = (int)cdiv(rows, ROW_WARPS);
-    // This chunk's rows in the group's dlogits block.
-    __nv_bfloat16* dlog_c = dlog + (size_t)(c % L.G) * L.C * L.Vp;
-
-    {
-      ProfScope ps(K_PREP, st, 0.0, (double)rows * K * 20.0 + rows * (NT + 1) * 2.0);
-      k_prep_teacher<<<row_blocks, ROW_WARPS * 32, 0, st>>>(
-          topk_idx + row0 * K, topk_logit + row0 * K, mask_c, rows, K, V, (int)NT, invT, sid, sp,
-          zs, tstart, plogp, ctl);
+    // Sources and destinations of this chunk: the caller's rows directly, or
+    // the staging buffers the listed rows are gathered into.
+    const void* h_c;
+    const int32_t* ids_c;
+    const float* lg_c;
+    const uint8_t* mask_c;
+    float* rl_c;
+    float* dH_c;
+    if (list) {
+      __nv_bfloat16* hdst = hstage + (size_t)(c % G) * L.C * L.H;
+      {
+        ProfScope ps(K_GATHER, st, 0.0, (double)rows * (L.H * 4.0 + K * 16.0 + 5.0));
+        k_gather_rows<<<rows, 128, 0, st>>>(q.rows + row0, rows, L.N, H, K,
+                                            static_cast<const __nv_bfloat16*>(q.hidden),
+                                            q.topk_idx, q.topk_logit, hdst, idstage, lgstage,
+                                            mstage);
+      }
+      h_c = hdst; ids_c = idstage; lg_c = lgstage; mask_c = mstage; rl_c = rlstage;
+      dH_c = dhstage;
+    } else {
+      h_c = static_cast<const uint8_t*>(q.hidden) + (size_t)row0 * L.H * 2;
+      ids_c = q.topk_idx ? q.topk_idx + row0 * K : nullptr;
+      lg_c = q.topk_logit ? q.topk_logit + row0 * K : nullptr;
+      mask_c = q.row_mask ? q.row_mask + row0 : nullptr;
+      rl_c = rl + row0;
+      dH_c = bwd ? q.dH + row0 * L.H : nullptr;
     }
+    // This chunk's rows in the group's dlogits block.
+    __nv_bfloat16* dlog_c = dlog + (size_t)(c % G) * L.C * L.Vp;
 
     CUtensorMap mapH_k;
     if (!make_map(&mapH_k, h_c, L.H, rows, L.H * 2, BK, CM)) return FCKL_ERR_CUDA;
-
-    // Forward: z = h W^T tiles, vocab-major units so concurrent pairs share W tiles.
+    // Forward units are vocab-major so that concurrent pairs share W tiles.
     SchedArgs sa_v{MT * NT, SCHED_VOCAB_MAJOR, (int)MT, (int)NT, (int)KBh, 1, 0};
     const int Gv = grid_for(MT * NT);
-    EpiLse::Params pf{rows, V, K, (int)NT, scale2, sid, tstart, zs, part};
+    const double gemm_flops = 2.0 * rows * (double)L.V * (double)L.H;
+
+    if (ent) {  // student entropy: forward GEMM with the entropy epilogue, then merge
+      EpiEntropy::Params pe{rows, V, 1, (int)NT, scale2, nullptr, nullptr, nullptr, part, upart};
+      {
+        ProfScope ps(K_ENT, st, gemm_flops, 2.0 * (rows + (double)L.V) * L.H + rows * NT * 12.0);
+        gemm_pair_kernel<EpiEntropy, false, false>
+            <<<Gv, GEMM_THREADS, pair_smem_bytes<EpiEntropy>(), st>>>(mapH_k, mapW_k, mapW_k, pe,
+                                                                      sa_v, ca);
+      }
+      {
+        ProfScope ps(K_ENT_MERGE, st, 0.0, rows * NT * 12.0 + rows * 5.0);
+        k_merge_entropy<<<row_blocks, ROW_WARPS * 32, 0, st>>>(part, upart, (int)NT, rows, mask_c,
+                                                               q.entropy + row0);
+      }
+      continue;
+    }
+
+    {
+      ProfScope ps(K_PREP, st, 0.0, (double)rows * K * 20.0 + rows * (NT + 1) * 2.0);
+      k_prep_teacher<<<row_blocks, ROW_WARPS * 32, 0, st>>>(ids_c, lg_c, mask_c, rows, K, V,
+                                                            (int)NT, invT, sid, sp, zs, tstart,
+                                                            plogp, ctl);
+    }
+    EpiLse::Params pf{rows, V, K, (int)NT, scale2, sid, tstart, zs, part, nullptr};
     CtlArgs ca_f = ca;
     ca_f.debug_skip_commit = (c == 0) ? ca.debug_skip_commit : 0;
-    const double gemm_flops = 2.0 * rows * (double)L.V * (double)L.H;
     {
       ProfScope ps(K_FWD, st, gemm_flops, 2.0 * (rows + (double)L.V) * L.H + rows * NT * 8.0);
       gemm_pair_kernel<EpiLse, false, false>
@@ -325,9 +434,16 @@ fckl_status run(bool bwd, const fckl_problem* prob, const void* hidden, const vo
     {
       ProfScope ps(K_MERGE, st, 0.0, (double)rows * K * 8.0 + rows * NT * 8.0 + rows * 13.0);
       k_merge_loss<<<row_blocks, ROW_WARPS * 32, 0, st>>>(part, (int)NT, rows, K, invT, zs, sp,
-                                                           plogp, mask_c, lse2, rl + row0);
+                                                           plogp, mask_c, lse2, rl_c);
     }
-    if (!bwd) continue;
+    if (!bwd) {
+      if (list) {
+        ProfScope ps(K_SCATTER, st, 0.0, rows * 12.0);
+        k_scatter_rows<<<rows, 128, 0, st>>>(q.rows + row0, rows, L.N, H, rlstage, rl, nullptr,
+                                             nullptr);
+      }
+      continue;
+    }
 
     // Backward 1: recompute the tiles and form bf16 dlogits = q - p~.
     EpiDlogits::Params pb{rows, V, K, (int)NT, scale2, lse2, sid, tstart, sp, mask_c};
@@ -341,11 +457,10 @@ fckl_status run(bool bwd, const fckl_problem* prob, const void* hidden, const vo
     }
 
     // Backward 2: dH[rows] = alpha * dlogits W; A = dlogits (K-major), B = W (MN-major).
-    if (cudaMemsetAsync(dH + row0 * L.H, 0, (size_t)rows * L.H * 4, st) != cudaSuccess)
-      return FCKL_ERR_CUDA;
+    if (cudaMemsetAsync(dH_c, 0, (size_t)rows * L.H * 4, st) != cudaSuccess) return FCKL_ERR_CUDA;
     CUtensorMap mapD_k, mapD_mn, mapH_mn, mapdH;
     if (!make_map(&mapD_k, dlog_c, L.V, rows, L.Vp * 2, BK, CM)) return FCKL_ERR_CUDA;
-    if (!make_map(&mapdH, dH + row0 * L.H, L.H, rows, L.H * 4, 32, 32, true)) return FCKL_ERR_CUDA;
+    if (!make_map(&mapdH, dH_c, L.H, rows, L.H * 4, 32, 32, true)) return FCKL_ERR_CUDA;
     const long long tiles_h = MT * NTh;
     const int S = choose_split(tiles_h, KBv, pairs);
     SchedArgs sa_h{tiles_h * S, SCHED_SPLIT_K, (int)MT, (int)NTh, (int)KBv, S, (int)tiles_h};
@@ -357,15 +472,21 @@ fckl_status run(bool bwd, const fckl_problem* prob, const void* hidden, const vo
           <<<grid_for(tiles_h * S), GEMM_THREADS, pair_smem_bytes<EpiDH>(), st>>>(
               mapD_k, mapW_mn, mapdH, ph, sa_h, ca);
     }
+    if (list) {
+      ProfScope ps(K_SCATTER, st, 0.0, rows * (12.0 + 8.0 * L.H));
+      k_scatter_rows<<<rows, 128, 0, st>>>(q.rows + row0, rows, L.N, H, rlstage, rl, dhstage,
+                                           q.dH);
+    }
 
     // Backward 3, once per group of G chunks (or at the last chunk):
     // dW (+)= alpha * dlogits^T h over the group's rows; A = dlogits^T, B = h
     // (both MN-major).
-    if ((c + 1) % L.G != 0 && c + 1 != L.nchunks) continue;
-    const long long g0 = c / L.G * L.G;  // first chunk of the group
+    if ((c + 1) % G != 0 && c + 1 != nchunks) continue;
+    const long long g0 = c / G * G;  // first chunk of the group
     const long long grow0 = g0 * L.C;
     const int grows = (int)(row0 + rows - grow0);
-    const void* h_g = static_cast<const uint8_t*>(hidden) + (size_t)grow0 * L.H * 2;
+    const void* h_g = list ? static_cast<const void*>(hstage)
+                           : static_cast<const uint8_t*>(q.hidden) + (size_t)grow0 * L.H * 2;
     if (!make_map(&mapD_mn, dlog, L.V, grows, L.Vp * 2, 64, BK)) return FCKL_ERR_CUDA;
     if (!make_map(&mapH_mn, h_g, L.H, grows, L.H * 2, 64, BK)) return FCKL_ERR_CUDA;
     const long long tiles_w = cdiv(L.V, PM) * NTh;
@@ -380,9 +501,9 @@ fckl_status run(bool bwd, const fckl_problem* prob, const void* hidden, const vo
               mapD_mn, mapH_mn, mapdW, pw, sa_w, ca);
     }
   }
-  {
+  if (!ent) {
     ProfScope ps(K_FINAL, st, 0.0, (double)L.N * 4.0);
-    k_finalize<<<1, 1024, 0, st>>>(rl, L.N, ctl, loss);
+    k_finalize<<<1, 1024, 0, st>>>(rl, L.N, ctl, q.loss);
   }
   if (cudaGetLastError() != cudaSuccess) return FCKL_ERR_CUDA;
   return FCKL_OK;
@@ -449,8 +570,14 @@ fckl_status fckl_fwd_noalloc(const fckl_problem* prob, const void* hidden, const
   }
   void* scratch = static_scratch();
   if (scratch == nullptr) return FCKL_ERR_CUDA;
-  const fckl_status st = run(false, &q, hidden, W, topk_idx, topk_logit, row_mask, loss, row_loss,
-                             nullptr, nullptr, scratch, kStaticScratchBytes, stream, true);
+  Request rq;
+  rq.mode = Mode::kFwd;
+  rq.prob = &q;
+  rq.hidden = hidden; rq.W = W; rq.topk_idx = topk_idx; rq.topk_logit = topk_logit;
+  rq.row_mask = row_mask; rq.loss = loss; rq.row_loss = row_loss;
+  rq.workspace = scratch; rq.ws_bytes = kStaticScratchBytes; rq.stream = stream;
+  rq.full_layout = false;
+  const fckl_status st = run(rq);
   if (st != FCKL_OK || device_status == nullptr) return st;
   k_export_status<<<1, 1, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       reinterpret_cast<const DeviceCtl*>(scratch), device_status);
@@ -472,16 +599,68 @@ fckl_status fckl_fwd(const fckl_problem* prob, const void* hidden, const void* W
                      const int32_t* topk_idx, const float* topk_logit, const uint8_t* row_mask,
                      float* loss, float* row_loss, void* workspace, size_t workspace_bytes,
                      void* stream) {
-  return run(false, prob, hidden, W, topk_idx, topk_logit, row_mask, loss, row_loss, nullptr,
-             nullptr, workspace, workspace_bytes, stream);
+  Request q;
+  q.mode = Mode::kFwd;
+  q.prob = prob; q.hidden = hidden; q.W = W; q.topk_idx = topk_idx; q.topk_logit = topk_logit;
+  q.row_mask = row_mask; q.loss = loss; q.row_loss = row_loss;
+  q.workspace = workspace; q.ws_bytes = workspace_bytes; q.stream = stream;
+  return run(q);
 }
 
 fckl_status fckl_fwd_bwd(const fckl_problem* prob, const void* hidden, const void* W,
                          const int32_t* topk_idx, const float* topk_logit,
                          const uint8_t* row_mask, float* loss, float* row_loss, float* dH,
                          float* dW, void* workspace, size_t workspace_bytes, void* stream) {
-  return run(true, prob, hidden, W, topk_idx, topk_logit, row_mask, loss, row_loss, dH, dW,
-             workspace, workspace_bytes, stream);
+  Request q;
+  q.mode = Mode::kFwdBwd;
+  q.prob = prob; q.hidden = hidden; q.W = W; q.topk_idx = topk_idx; q.topk_logit = topk_logit;
+  q.row_mask = row_mask; q.loss = loss; q.row_loss = row_loss; q.dH = dH; q.dW = dW;
+  q.workspace = workspace; q.ws_bytes = workspace_bytes; q.stream = stream;
+  return run(q);
+}
+
+fckl_status fckl_fwd_bwd_rows(const fckl_problem* prob, const void* hidden, const void* W,
+                              const int32_t* topk_idx, const float* topk_logit,
+                              const int32_t* rows, int64_t n_rows, float* loss, float* row_loss,
+                              float* dH, float* dW, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+  if (rows == nullptr || (dH == nullptr) != (dW == nullptr)) return FCKL_ERR_INVALID_ARG;
+  Request q;
+  q.mode = dH ? Mode::kFwdBwd : Mode::kFwd;
+  q.prob = prob; q.hidden = hidden; q.W = W; q.topk_idx = topk_idx; q.topk_logit = topk_logit;
+  q.rows = rows; q.n_rows = n_rows;
+  q.loss = loss; q.row_loss = row_loss; q.dH = dH; q.dW = dW;
+  q.workspace = workspace; q.ws_bytes = workspace_bytes; q.stream = stream;
+  return run(q);
+}
+
+fckl_status fckl_student_entropy(const fckl_problem* prob, const void* hidden, const void* W,
+                                 const uint8_t* row_mask, float* row_entropy, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  if (prob == nullptr) return FCKL_ERR_INVALID_ARG;
+  fckl_problem p1 = *prob;  // the teacher does not take part: K is ignored
+  p1.K = 1;
+  Request q;
+  q.mode = Mode::kEntropy;
+  q.prob = &p1; q.hidden = hidden; q.W = W; q.row_mask = row_mask; q.entropy = row_entropy;
+  q.workspace = workspace; q.ws_bytes = workspace_bytes; q.stream = stream;
+  return run(q);
+}
+
+fckl_status fckl_select_top_rows(const float* score, const uint8_t* row_mask, int64_t N,
+                                 int64_t n_select, int32_t* rows_out, int32_t* count_out,
+                                 void* stream) {
+  if (!score || !rows_out || !count_out || N < 1 || N > INT32_MAX || n_select < 1 ||
+      n_select > N || !aligned(score, 4) || !aligned(rows_out, 4) || !aligned(count_out, 4))
+    return FCKL_ERR_INVALID_ARG;
+  const DeviceInfo* dev = device_info();
+  if (dev == nullptr || !dev->ok) return FCKL_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  {
+    ProfScope ps(K_SELECT, st, 0.0, N * 5.0 * 4 + n_select * 4.0);
+    k_select_top_rows<<<1, 1024, 0, st>>>(score, row_mask, N, n_select, rows_out, count_out);
+  }
+  return cudaGetLastError() == cudaSuccess ? FCKL_OK : FCKL_ERR_CUDA;
 }
 
 fckl_status fckl_check(void* workspace, void* stream) {

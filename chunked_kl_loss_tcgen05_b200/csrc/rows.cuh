@@ -4,6 +4,8 @@
 
 #include <climits>
 
+#include <cuda_bf16.h>
+
 #include "gemm.cuh"
 
 namespace fckl {
@@ -42,6 +44,182 @@ __global__ void __launch_bounds__(1024) k_count_valid(const uint8_t* __restrict_
     for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
     if (threadIdx.x == 0) ctl->n_valid = c;
   }
+}
+
+// N_valid for a row list: entries in [0, N) count; negative entries are
+// padding and are skipped; entries >= N are reported as bad indices.  One block.
+__global__ void __launch_bounds__(1024) k_count_list(const int32_t* __restrict__ rows, long long n,
+                                                     long long N, DeviceCtl* ctl) {
+  __shared__ int red[32];
+  int c = 0;
+  bool bad = false;
+  for (long long i = threadIdx.x; i < n; i += blockDim.x) {
+    const int r = rows[i];
+    c += (r >= 0 && r < N);
+    bad |= r >= N;
+  }
+  if (__syncthreads_or(bad) && threadIdx.x == 0) atomicOr(&ctl->err, kErrBadIndex);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = c;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    c = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+    if (threadIdx.x == 0) ctl->n_valid = c;
+  }
+}
+
+// Gather the listed rows of one chunk (block i copies list entry i): hidden
+// row -> hst[i] (bf16, 16-byte vectors), teacher ids/logits -> idst/lgst[i],
+// mst[i] = 1.  Entries outside [0, N) give a zero row with mst[i] = 0.
+__global__ void __launch_bounds__(128)
+    k_gather_rows(const int32_t* __restrict__ list, int rows_c, long long N, int H, int K,
+                  const __nv_bfloat16* __restrict__ hidden, const int32_t* __restrict__ ids,
+                  const float* __restrict__ lg, __nv_bfloat16* __restrict__ hst,
+                  int32_t* __restrict__ idst, float* __restrict__ lgst, uint8_t* __restrict__ mst) {
+  const int i = blockIdx.x;
+  if (i >= rows_c) return;
+  const int r = list[i];
+  const bool ok = r >= 0 && r < N;
+  const uint4* src = reinterpret_cast<const uint4*>(hidden + (size_t)(ok ? r : 0) * H);
+  uint4* dst = reinterpret_cast<uint4*>(hst + (size_t)i * H);
+  for (int j = threadIdx.x; j < H / 8; j += blockDim.x)
+    dst[j] = ok ? src[j] : make_uint4(0u, 0u, 0u, 0u);
+  for (int k = threadIdx.x; k < K; k += blockDim.x) {
+    idst[(size_t)i * K + k] = ok ? ids[(size_t)r * K + k] : 0;
+    lgst[(size_t)i * K + k] = ok ? lg[(size_t)r * K + k] : 0.f;
+  }
+  if (threadIdx.x == 0) mst[i] = ok ? 1 : 0;
+}
+
+// Scatter one chunk's per-entry results back to the listed rows: row loss and
+// (when dH is given) the fp32 dH row.
+__global__ void __launch_bounds__(128)
+    k_scatter_rows(const int32_t* __restrict__ list, int rows_c, long long N, int H,
+                   const float* __restrict__ rl_stage, float* __restrict__ rl,
+                   const float* __restrict__ dh_stage, float* __restrict__ dH) {
+  const int i = blockIdx.x;
+  if (i >= rows_c) return;
+  const int r = list[i];
+  if (r < 0 || r >= N) return;
+  if (threadIdx.x == 0) rl[r] = rl_stage[i];
+  if (dH == nullptr) return;
+  const float4* src = reinterpret_cast<const float4*>(dh_stage + (size_t)i * H);
+  float4* dst = reinterpret_cast<float4*>(dH + (size_t)r * H);
+  for (int j = threadIdx.x; j < H / 4; j += blockDim.x) dst[j] = src[j];
+}
+
+// Order-preserving map of a float to uint32 (larger float -> larger key).
+__device__ __forceinline__ uint32_t float_key(float f) {
+  const uint32_t b = __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// Exclusive block-wide prefix sum of one int per thread (blockDim.x = 1024).
+__device__ __forceinline__ int block_exclusive_scan(int v, int* sh, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sh[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < (int)(blockDim.x >> 5) ? sh[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    sh[lane] = w;  // inclusive warp totals
+  }
+  __syncthreads();
+  const int before = (warp > 0 ? sh[warp - 1] : 0) + x - v;
+  *total = sh[(blockDim.x >> 5) - 1];
+  __syncthreads();
+  return before;
+}
+
+// Top-n rows by score among valid rows (row_mask != 0, or all), one block:
+// an MSB-first radix select (8 bits per pass) finds the n-th largest key, then
+// every row above it and the lowest-index rows equal to it are written to
+// rows_out in ascending row order.  n = min(n_select, valid rows); the rest of
+// rows_out[0, n_select) is set to -1 and *count_out = n.
+__global__ void __launch_bounds__(1024)
+    k_select_top_rows(const float* __restrict__ score, const uint8_t* __restrict__ mask,
+                      long long N, long long n_select, int32_t* __restrict__ rows_out,
+                      int32_t* __restrict__ count_out) {
+  __shared__ int hist[256];
+  __shared__ int sh[32];
+  __shared__ uint32_t s_prefix, s_need;
+  const int tid = threadIdx.x;
+  // number of valid rows
+  int cnt = 0;
+  for (long long i = tid; i < N; i += blockDim.x) cnt += (mask == nullptr || mask[i] != 0);
+  int nvalid = 0;
+  block_exclusive_scan(cnt, sh, &nvalid);
+  const long long n = n_select < nvalid ? n_select : nvalid;
+  uint32_t prefix = 0, need = (uint32_t)n;  // need: how many keys >= threshold still to take
+  if (n > 0) {
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
+      const uint32_t hi_mask = pass == 0 ? 0u : (0xFFFFFFFFu << (32 - 8 * pass));
+      for (int b = tid; b < 256; b += blockDim.x) hist[b] = 0;
+      __syncthreads();
+      for (long long i = tid; i < N; i += blockDim.x) {
+        if (mask != nullptr && mask[i] == 0) continue;
+        const uint32_t k = float_key(score[i]);
+        if ((k & hi_mask) == (prefix & hi_mask)) atomicAdd(&hist[(k >> shift) & 255u], 1);
+      }
+      __syncthreads();
+      if (tid == 0) {
+        uint32_t acc = 0;
+        int b = 255;
+        for (; b > 0; --b) {  // walk bins from the largest digit down
+          if (acc + (uint32_t)hist[b] >= need) break;
+          acc += (uint32_t)hist[b];
+        }
+        s_prefix = prefix | ((uint32_t)b << shift);
+        s_need = need - acc;
+      }
+      __syncthreads();
+      prefix = s_prefix;
+      need = s_need;
+      __syncthreads();
+    }
+  }
+  // prefix = threshold key; need = how many rows equal to it are taken.
+  const long long per = (N + blockDim.x - 1) / blockDim.x;
+  const long long i0 = tid * per, i1 = (i0 + per < N) ? i0 + per : N;
+  int n_gt = 0, n_eq = 0;
+  if (n > 0)
+    for (long long i = i0; i < i1; ++i) {
+      if (mask != nullptr && mask[i] == 0) continue;
+      const uint32_t k = float_key(score[i]);
+      n_gt += k > prefix;
+      n_eq += k == prefix;
+    }
+  int tot;
+  const int eq_before = block_exclusive_scan(n_eq, sh, &tot);
+  int take_eq = 0;
+  if (eq_before < (int)need) take_eq = min(n_eq, (int)need - eq_before);
+  const int out_before = block_exclusive_scan(n_gt + take_eq, sh, &tot);
+  if (n > 0) {
+    int pos = out_before, eq_seen = 0;
+    for (long long i = i0; i < i1; ++i) {
+      if (mask != nullptr && mask[i] == 0) continue;
+      const uint32_t k = float_key(score[i]);
+      bool take = k > prefix;
+      if (k == prefix) take = eq_seen++ < take_eq;
+      if (take && pos < n_select) rows_out[pos++] = (int32_t)i;
+    }
+  }
+  for (long long j = n + tid; j < n_select; j += blockDim.x) rows_out[j] = -1;
+  if (tid == 0) *count_out = (int32_t)n;
 }
 
 // Teacher side of one chunk, one warp per row: p = softmax(topk_logit / T)
@@ -169,6 +347,38 @@ __global__ void __launch_bounds__(ROW_WARPS * 32)
     const bool keep = mask == nullptr || mask[row] != 0;
     lse2_out[row] = L2;
     row_loss[row] = keep ? plogp[row] - acc : 0.f;
+  }
+}
+
+// Student entropy per row from the per-tile (max, sum, weighted sum) partials:
+// with a = z log2(e) / T, S = sum 2^(a - M), U = sum 2^(a - M) a and
+// LSE2 = M + log2 S, H(q) = -sum q ln q = ln2 * (LSE2 - U / S) nats.
+// Masked rows get 0.
+__global__ void __launch_bounds__(ROW_WARPS * 32)
+    k_merge_entropy(const float2* __restrict__ partials, const float* __restrict__ upart, int NT,
+                    int rows_c, const uint8_t* __restrict__ mask, float* __restrict__ entropy) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * ROW_WARPS + warp;
+  if (row >= rows_c) return;
+  const float2* pr = partials + (size_t)row * NT;
+  const float* pu = upart + (size_t)row * NT;
+  float M = -INFINITY;
+  for (int t = lane; t < NT; t += 32) M = fmaxf(M, pr[t].x);
+  M = warp_max(M);
+  float S = 0.f, U = 0.f;
+  for (int t = lane; t < NT; t += 32) {
+    const float2 q = pr[t];
+    if (q.x > -INFINITY) {
+      const float f = exp2f(q.x - M);
+      S += q.y * f;
+      U += pu[t] * f;
+    }
+  }
+  S = warp_sum(S);
+  U = warp_sum(U);
+  if (lane == 0) {
+    const bool keep = mask == nullptr || mask[row] != 0;
+    entropy[row] = keep ? 0.69314718055994530942f * (M + log2f(S) - U / S) : 0.f;
   }
 }
 

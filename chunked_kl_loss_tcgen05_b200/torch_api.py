@@ -13,7 +13,8 @@ import torch
 from . import (FcklError, FcklProblem, FCKL_OK, fckl_check, fckl_fwd, fckl_fwd_bwd,
                fckl_workspace_bytes)
 
-__all__ = ["make_problem", "alloc_workspace", "fused_kl_fwd", "fused_kl_fwd_bwd",
+__all__ = ["make_problem", "alloc_workspace", "fused_kl_fwd", "fused_kl_fwd_bwd", "student_entropy",
+           "select_top_rows", "fused_kl_rows", "arrays_to_device",
            "fused_kl_from_host", "FusedChunkedKL", "fused_chunked_kl_loss"]
 
 
@@ -164,3 +165,70 @@ def arrays_to_device(hidden_bits, W_bits, topk_idx, topk_logit, row_mask, device
            t(topk_logit, np.float32).to(device),
            None if row_mask is None else t(row_mask, np.uint8).to(device)]
     return tuple(out)
+
+
+def student_entropy(hidden, W, row_mask=None, T=1.0, chunk=0, workspace=None, check=True):
+    """Per-row student entropy H(softmax(W h / T)) in nats, [N] fp32 (0 for masked rows)."""
+    from . import fckl_student_entropy
+    hidden, W = _bits(hidden), _bits(W)
+    N, H = hidden.shape
+    prob = FcklProblem(N, H, W.shape[0], 1, T, chunk)
+    dev = hidden.device
+    if workspace is None:
+        workspace = alloc_workspace(prob, dev)
+    ent = torch.empty(N, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    st = fckl_student_entropy(prob, hidden.data_ptr(), W.data_ptr(),
+                              None if row_mask is None else row_mask.data_ptr(), ent.data_ptr(),
+                              workspace.data_ptr(), workspace.numel(), stream)
+    if st != FCKL_OK:
+        raise FcklError(st, "fckl_student_entropy")
+    if check:
+        st = fckl_check(workspace.data_ptr(), stream)
+        if st != FCKL_OK:
+            raise FcklError(st, "fckl_check")
+    return ent
+
+
+def select_top_rows(score, n_select, row_mask=None):
+    """(rows int32 [n_select] ascending, padded with -1; count int32 [1]) on device."""
+    from . import fckl_select_top_rows
+    N = score.numel()
+    rows = torch.empty(n_select, dtype=torch.int32, device=score.device)
+    count = torch.empty(1, dtype=torch.int32, device=score.device)
+    st = fckl_select_top_rows(score.data_ptr(), None if row_mask is None else row_mask.data_ptr(),
+                              N, n_select, rows.data_ptr(), count.data_ptr(),
+                              torch.cuda.current_stream(score.device).cuda_stream)
+    if st != FCKL_OK:
+        raise FcklError(st, "fckl_select_top_rows")
+    return rows, count
+
+
+def fused_kl_rows(hidden, W, topk_idx, topk_logit, rows, T=1.0, chunk=0, workspace=None,
+                  grads=True, want_row_loss=False, check=True):
+    """Loss (and dH, dW) over the listed rows only.  Returns (loss, row_loss, dH, dW)."""
+    from . import fckl_fwd_bwd_rows
+    hidden, W = _bits(hidden), _bits(W)
+    _check_inputs(hidden, W, topk_idx, topk_logit, None)
+    prob = make_problem(hidden, W, topk_idx, T, chunk)
+    dev = hidden.device
+    if workspace is None:
+        workspace = alloc_workspace(prob, dev)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    row_loss = torch.empty(prob.N, dtype=torch.float32, device=dev) if want_row_loss else None
+    dH = torch.empty(prob.N, prob.H, dtype=torch.float32, device=dev) if grads else None
+    dW = torch.empty(prob.V, prob.H, dtype=torch.float32, device=dev) if grads else None
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    st = fckl_fwd_bwd_rows(prob, hidden.data_ptr(), W.data_ptr(), topk_idx.data_ptr(),
+                           topk_logit.data_ptr(), rows.data_ptr(), rows.numel(), loss.data_ptr(),
+                           None if row_loss is None else row_loss.data_ptr(),
+                           None if dH is None else dH.data_ptr(),
+                           None if dW is None else dW.data_ptr(), workspace.data_ptr(),
+                           workspace.numel(), stream)
+    if st != FCKL_OK:
+        raise FcklError(st, "fckl_fwd_bwd_rows")
+    if check:
+        st = fckl_check(workspace.data_ptr(), stream)
+        if st != FCKL_OK:
+            raise FcklError(st, "fckl_check")
+    return loss, row_loss, dH, dW

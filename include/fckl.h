@@ -94,8 +94,11 @@ typedef struct {
   int64_t chunk;  /* rows per chunk, 0 = auto     */
 } fckl_problem;
 
-/* Bytes of device workspace fckl_fwd / fckl_fwd_bwd need for `prob` (0 when the
- * problem is invalid).  Pure host arithmetic; needs no GPU. */
+/* Bytes of device workspace fckl_fwd / fckl_fwd_bwd / fckl_fwd_bwd_rows /
+ * fckl_student_entropy need for `prob` (0 when the problem is invalid): the
+ * per-chunk teacher, log-sum-exp and dlogits buffers, N floats of row loss
+ * and the staging buffers row-list calls gather into.  Pure host arithmetic;
+ * needs no GPU. */
 size_t fckl_workspace_bytes(const fckl_problem* prob);
 
 /* The chunk size the library will use for `prob` (resolves chunk = 0), or -1
@@ -154,6 +157,50 @@ fckl_status fckl_fwd_noalloc(const fckl_problem* prob, const void* hidden, const
                              const uint8_t* row_mask, float* loss, float* row_loss,
                              int32_t* device_status, void* stream);
 
+/* ----------------------------------------------------------------------------
+ * Position selection by student entropy (the selective-distillation method of
+ * "기술 요약: 선택적 지식 증류(Selective Knowledge Distillation)의 재고", sections
+ * 방법론 (SE-KD: supervise the top-k% positions by student entropy H(q_t)) and
+ * 효율성 최적화 (chunked entropy computation; a selective LM head that
+ * computes logits and gradients only at the selected positions)).
+ * ------------------------------------------------------------------------- */
+
+/* Student entropy H(q_r) = -sum_v q_v ln q_v (nats), q = softmax(W h_r / T), for
+ * every row, written to row_entropy [N] (0 for masked rows).  Computed chunk by
+ * chunk in the epilogue of the projection GEMM: the logits are never stored.
+ * prob->K and the teacher arrays take no part (K is ignored).  Uses the same
+ * workspace as fckl_fwd_bwd.  Cost: 2*H*V flops per row. */
+fckl_status fckl_student_entropy(const fckl_problem* prob, const void* hidden, const void* W,
+                                 const uint8_t* row_mask, float* row_entropy, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
+/* The n_select rows with the largest score (e.g. row_entropy) among the valid
+ * rows (row_mask != 0, or all rows when NULL), written to rows_out in
+ * ascending row order; ties at the threshold go to the lower row index.  If
+ * fewer than n_select rows are valid, all valid rows are written and the rest
+ * of rows_out[0, n_select) is set to -1.  *count_out (device int32) receives
+ * the number of rows written.  Scores must not be NaN.  Device pointers;
+ * 1 <= n_select <= N.  One kernel, no workspace. */
+fckl_status fckl_select_top_rows(const float* score, const uint8_t* row_mask, int64_t N,
+                                 int64_t n_select, int32_t* rows_out, int32_t* count_out,
+                                 void* stream);
+
+/* Loss and gradients over a list of rows only (a selective LM head): rows is a
+ * device int32 [n_rows] of distinct row indices in [0, N); negative entries are
+ * skipped (so the padded output of fckl_select_top_rows can be passed as is).
+ * The listed rows are gathered chunk by chunk, so the GEMM work scales with
+ * the number of listed rows, not with N.  Results equal fckl_fwd_bwd with
+ * row_mask = the indicator of the listed rows: loss = mean over listed rows,
+ * row_loss and dH rows of unlisted rows are 0, dW sums over listed rows.
+ * dH = dW = NULL computes the loss only.  hidden/topk arrays are the full
+ * [N, ...] arrays; the workspace is fckl_workspace_bytes(prob).  An entry >= N
+ * is reported by fckl_check as FCKL_ERR_BAD_INDEX and skipped. */
+fckl_status fckl_fwd_bwd_rows(const fckl_problem* prob, const void* hidden, const void* W,
+                              const int32_t* topk_idx, const float* topk_logit,
+                              const int32_t* rows, int64_t n_rows, float* loss, float* row_loss,
+                              float* dH, float* dW, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
 /* Synchronises `stream`, then returns the first device-side error recorded in
  * `workspace` by the last call that used it (FCKL_OK if none), or
  * FCKL_ERR_CUDA if the stream reports a CUDA error. */
@@ -174,7 +221,8 @@ const char* fckl_status_string(fckl_status status);
  * many kinds were seen, or -1 on a CUDA error.  Recording is process-wide and
  * not thread-safe.
  * Kinds: 0 count_valid, 1 prep_teacher, 2 fwd_logits_lse, 3 merge_loss,
- *        4 bwd_dlogits, 5 dH_gemm, 6 dW_gemm, 7 finalize. */
+ *        4 bwd_dlogits, 5 dH_gemm, 6 dW_gemm, 7 finalize, 8 entropy_gemm,
+ *        9 merge_entropy, 10 gather_rows, 11 scatter_rows, 12 select_rows. */
 typedef struct {
   char name[32];     /* kernel kind, e.g. "fwd_logits_lse" */
   int64_t launches;  /* launches recorded */

@@ -20,3 +20,4 @@ from .kl import (  # noqa: F401
     widen_bf16,
     oracle_from_inputs,
 )
+from .selective import student_entropy, select_top_rows  # noqa: F401

@@ -1,0 +1,116 @@
+"""GPU parity of the selective-distillation path: student entropy, top-n row
+selection and the loss over selected rows only, against the fp64 oracle.
+Tolerances as in test_gpu_parity: 1e-3 relative on losses and entropies,
+2e-2 relative Frobenius on gradients; row selection is index work and must
+match exactly."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from chunked_kl_loss_tcgen05_b200 import FCKL_ERR_BAD_INDEX, FcklError
+from chunked_kl_loss_tcgen05_b200.torch_api import (arrays_to_device, fused_kl_fwd_bwd,
+                                                    fused_kl_rows, select_top_rows,
+                                                    student_entropy)
+
+pytestmark = pytest.mark.gpu
+
+RTOL = 1e-3
+GRAD_RTOL = 2e-2
+
+
+def rel_fro(a, b):
+    a = np.asarray(a, np.float64); b = np.asarray(b, np.float64)
+    return np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300)
+
+
+@pytest.mark.parametrize("shape", [(256, 256, 4096, 1.0, 64), (333, 200, 1003, 1.7, 128),
+                                   (1000, 64, 513, 0.5, 0)])
+def test_entropy_matches_oracle(shape):
+    N, H, V, T, chunk = shape
+    inp = synth.make_custom(N, H, V, 4, T=T, mask_frac=0.1, seed=31 + N)
+    d = arrays_to_device(inp.hidden, inp.W, inp.topk_idx, inp.topk_logit, inp.row_mask)
+    e = student_entropy(d[0], d[1], d[4], T=T, chunk=chunk).cpu().numpy()
+    ref = oracle.student_entropy(inp.hidden, inp.W, T, inp.row_mask)
+    np.testing.assert_allclose(e, ref, rtol=RTOL, atol=1e-4)
+
+
+def test_entropy_llama_shape_sampled_rows():
+    inp = synth.make_inputs(1)
+    rows = synth.sample_rows(inp, 64)
+    d = arrays_to_device(inp.hidden, inp.W, inp.topk_idx, inp.topk_logit, inp.row_mask)
+    e = student_entropy(d[0], d[1], d[4], T=inp.cfg.T).cpu().numpy()
+    _, ref = oracle.student_entropy(inp.hidden, inp.W, inp.cfg.T, inp.row_mask, rows=rows)
+    np.testing.assert_allclose(e[rows], ref, rtol=RTOL, atol=1e-4)
+    assert (e[inp.row_mask == 0] == 0).all()
+
+
+@pytest.mark.parametrize("N,n,ties", [(1, 1, False), (1000, 200, True), (100000, 20000, False),
+                                      (262144, 52429, True), (5000, 5000, False)])
+def test_select_matches_oracle(N, n, ties):
+    rng = np.random.default_rng(N + n)
+    score = (rng.integers(0, 50, N) * 0.25 if ties else rng.standard_normal(N) * 3).astype(np.float32)
+    mask = (rng.random(N) < 0.9).astype(np.uint8)
+    rows, count = select_top_rows(torch.from_numpy(score).cuda(), n, torch.from_numpy(mask).cuda())
+    ref, rcount = oracle.select_top_rows(score, mask, n)
+    assert count.item() == rcount
+    np.testing.assert_array_equal(rows.cpu().numpy(), ref)
+
+
+def _check_rows(inp, rows_np, T, chunk):
+    d = arrays_to_device(inp.hidden, inp.W, inp.topk_idx, inp.topk_logit, None)
+    rows = torch.from_numpy(rows_np.astype(np.int32)).cuda()
+    loss, rl, dH, dW = fused_kl_rows(d[0], d[1], d[2], d[3], rows, T=T, chunk=chunk,
+                                     want_row_loss=True)
+    torch.cuda.synchronize()
+    mask = np.zeros(inp.cfg.N, np.uint8)
+    mask[rows_np[rows_np >= 0]] = 1
+    o = oracle.fused_chunked_kl(inp.hidden, inp.W, inp.topk_idx, inp.topk_logit, mask, T)
+    assert abs(loss.item() - o["loss"]) <= RTOL * abs(o["loss"])
+    np.testing.assert_allclose(rl.cpu().numpy(), o["row_loss"], rtol=RTOL, atol=1e-4)
+    assert rel_fro(dH.cpu().numpy(), o["dH"]) <= GRAD_RTOL
+    assert rel_fro(dW.cpu().numpy(), o["dW"]) <= GRAD_RTOL
+    # the same as the masked full-row call
+    l2, _, dH2, dW2 = fused_kl_fwd_bwd(d[0], d[1], d[2], d[3], torch.from_numpy(mask).cuda(), T=T,
+                                       chunk=chunk)
+    assert abs(l2.item() - loss.item()) <= 1e-5 * abs(loss.item())
+    assert rel_fro(dH.cpu().numpy(), dH2.cpu().numpy()) < 1e-5
+    assert rel_fro(dW.cpu().numpy(), dW2.cpu().numpy()) < 1e-5
+
+
+@pytest.mark.parametrize("case", [(600, 128, 2000, 10, 1.0, 128, 0.2), (1000, 64, 513, 7, 2.0, 37, 0.5),
+                                  (300, 256, 4096, 16, 1.0, 0, 1.0)])
+def test_loss_over_listed_rows(case):
+    N, H, V, K, T, chunk, frac = case
+    inp = synth.make_custom(N, H, V, K, T=T, sigma=2.0, seed=41 + N)
+    rng = np.random.default_rng(N)
+    n = max(1, int(frac * N))
+    rows = np.sort(rng.choice(N, n, replace=False))
+    padded = np.concatenate([rows, -np.ones(7, np.int64)])  # padding entries are skipped
+    _check_rows(inp, padded, T, chunk)
+
+
+def test_sekd_pipeline_top_entropy_rows():
+    """Entropy -> top 20% rows -> loss and gradients over those rows."""
+    inp = synth.make_custom(2048, 256, 8192, 32, T=1.0, sigma=3.0, mask_frac=0.05, seed=55)
+    d = arrays_to_device(inp.hidden, inp.W, inp.topk_idx, inp.topk_logit, inp.row_mask)
+    e = student_entropy(d[0], d[1], d[4])
+    n = int(0.2 * 2048)
+    rows, count = select_top_rows(e, n, d[4])
+    e_ref = oracle.student_entropy(inp.hidden, inp.W, 1.0, inp.row_mask)
+    ref_rows, _ = oracle.select_top_rows(e.cpu().numpy(), inp.row_mask, n)
+    np.testing.assert_array_equal(rows.cpu().numpy(), ref_rows)   # selection of the GPU scores
+    top_ref, _ = oracle.select_top_rows(e_ref.astype(np.float32), inp.row_mask, n)
+    overlap = len(np.intersect1d(rows.cpu().numpy(), top_ref)) / n
+    assert overlap > 0.97                                          # near-ties may swap
+    _check_rows(inp, rows.cpu().numpy().astype(np.int64), 1.0, 0)
+
+
+def test_listed_row_out_of_range_is_reported():
+    inp = synth.make_custom(64, 64, 512, 8, seed=6)
+    d = arrays_to_device(inp.hidden, inp.W, inp.topk_idx, inp.topk_logit, None)
+    rows = torch.tensor([1, 5, 64, 9], dtype=torch.int32, device="cuda")
+    with pytest.raises(FcklError) as ei:
+        fused_kl_rows(d[0], d[1], d[2], d[3], rows)
+    assert ei.value.status == FCKL_ERR_BAD_INDEX
