@@ -17,7 +17,7 @@ import os
 __all__ = [
     "FCKL_OK", "FCKL_ERR_INVALID_ARG", "FCKL_ERR_UNSUPPORTED", "FCKL_ERR_WORKSPACE",
     "FCKL_ERR_BAD_INDEX", "FCKL_ERR_BAD_TEACHER", "FCKL_ERR_TIMEOUT", "FCKL_ERR_CUDA",
-    "FCKL_K_MAX", "FcklProblem", "FcklError", "load", "lib_path", "exported_symbols",
+    "FCKL_K_MAX", "FCKL_TEACHER_LOGITS", "FCKL_TEACHER_PROBS", "FcklProblem", "FcklError", "load", "lib_path", "exported_symbols",
     "fckl_workspace_bytes", "fckl_resolved_chunk", "fckl_fwd", "fckl_fwd_bwd", "fckl_check",
     "fckl_status_string", "FcklKernelStat", "fckl_profile_begin", "fckl_profile_end",
     "fckl_fwd_noalloc", "fckl_student_entropy", "fckl_select_top_rows", "fckl_fwd_bwd_rows",
@@ -42,13 +42,18 @@ exported_symbols = ("fckl_workspace_bytes", "fckl_resolved_chunk", "fckl_fwd", "
                     "fckl_fwd_bwd_rows")
 
 
+FCKL_TEACHER_LOGITS = 0
+FCKL_TEACHER_PROBS = 1
+
+
 class FcklProblem(ctypes.Structure):
     """Mirror of ``fckl_problem``."""
     _fields_ = [("N", ctypes.c_int64), ("H", ctypes.c_int64), ("V", ctypes.c_int64),
-                ("K", ctypes.c_int32), ("T", ctypes.c_float), ("chunk", ctypes.c_int64)]
+                ("K", ctypes.c_int32), ("T", ctypes.c_float), ("chunk", ctypes.c_int64),
+                ("teacher", ctypes.c_int32)]
 
-    def __init__(self, N, H, V, K, T=1.0, chunk=0):
-        super().__init__(int(N), int(H), int(V), int(K), float(T), int(chunk))
+    def __init__(self, N, H, V, K, T=1.0, chunk=0, teacher=FCKL_TEACHER_LOGITS):
+        super().__init__(int(N), int(H), int(V), int(K), float(T), int(chunk), int(teacher))
 
 
 class FcklKernelStat(ctypes.Structure):

@@ -42,6 +42,7 @@ bool valid_problem(const fckl_problem* p) {
   if (p->N < 1 || p->H < 1 || p->V < 1 || p->K < 1 || p->chunk < 0) return false;
   if (!(std::isfinite(p->T) && p->T > 0.f)) return false;
   if (p->N > INT32_MAX || p->H > INT32_MAX || p->V > INT32_MAX) return false;
+  if (p->teacher != FCKL_TEACHER_LOGITS && p->teacher != FCKL_TEACHER_PROBS) return false;
   return true;
 }
 
@@ -418,9 +419,9 @@ fckl_status run(const Request& q) {
 
     {
       ProfScope ps(K_PREP, st, 0.0, (double)rows * K * 20.0 + rows * (NT + 1) * 2.0);
-      k_prep_teacher<<<row_blocks, ROW_WARPS * 32, 0, st>>>(ids_c, lg_c, mask_c, rows, K, V,
-                                                            (int)NT, invT, sid, sp, zs, tstart,
-                                                            plogp, ctl);
+      k_prep_teacher<<<row_blocks, ROW_WARPS * 32, 0, st>>>(
+          ids_c, lg_c, mask_c, rows, K, V, (int)NT, invT, prob->teacher == FCKL_TEACHER_PROBS,
+          sid, sp, zs, tstart, plogp, ctl);
     }
     EpiLse::Params pf{rows, V, K, (int)NT, scale2, sid, tstart, zs, part, nullptr};
     CtlArgs ca_f = ca;

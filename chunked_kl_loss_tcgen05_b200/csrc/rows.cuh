@@ -222,20 +222,23 @@ __global__ void __launch_bounds__(1024)
   if (tid == 0) *count_out = (int32_t)n;
 }
 
-// Teacher side of one chunk, one warp per row: p = softmax(topk_logit / T)
-// over the K cached logits, sum_k p_k log p_k, the (id, p) pairs sorted by id,
-// and for every vocab tile of 256 columns the position of its first id in the
-// sorted list (tstart, NT + 1 entries per row), so that a GEMM epilogue finds
-// the cached ids of its tile with one load.  Ids outside [0, V) are recorded
-// as an error and replaced by INT_MAX, which no vocab column matches.
+// Teacher side of one chunk, one warp per row: the teacher probabilities of
+// the K cache entries (softmax of topk_logit / T, or given weights
+// normalised), the (id, p) pairs sorted by id, sum p~ log p~ over the distinct
+// ids (entries with the same id add into one class), and for every vocab tile
+// of 256 columns the position of its first id in the sorted list (tstart,
+// NT + 1 entries per row), so that a GEMM epilogue finds the cached ids of its
+// tile with one load.  Ids outside [0, V) are recorded as an error and replaced
+// by INT_MAX, which no vocab column matches.
 __global__ void __launch_bounds__(ROW_WARPS * 32)
     k_prep_teacher(const int32_t* __restrict__ ids, const float* __restrict__ lg,
                    const uint8_t* __restrict__ mask, int rows_c, int K, int V, int NT,
-                   float invT, int* __restrict__ sid, float* __restrict__ sp,
+                   float invT, bool probs, int* __restrict__ sid, float* __restrict__ sp,
                    float* __restrict__ zs, uint16_t* __restrict__ tstart,
                    float* __restrict__ plogp, DeviceCtl* ctl) {
   __shared__ int s_ids[ROW_WARPS][K_MAX];
   __shared__ int s_sorted[ROW_WARPS][K_MAX];
+  __shared__ float s_sp[ROW_WARPS][K_MAX];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * ROW_WARPS + warp;
   if (row >= rows_c) return;  // warp-uniform
@@ -247,14 +250,19 @@ __global__ void __launch_bounds__(ROW_WARPS * 32)
 #pragma unroll
   for (int i = 0; i < K_MAX / 32; ++i) {
     const int k = lane + 32 * i;
-    t[i] = -INFINITY;
+    t[i] = probs ? 0.f : -INFINITY;
     id[i] = INT_MAX;
     if (k < K) {
       const float x = lg[(size_t)row * K + k];
       int d = ids[(size_t)row * K + k];
-      if (isnan(x) || x == INFINITY) bad_val = true;
+      if (probs) {
+        if (!(x >= 0.f) || x == INFINITY) bad_val = true;  // negative, NaN or +inf weight
+        t[i] = (x >= 0.f && x < INFINITY) ? x : 0.f;
+      } else {
+        if (isnan(x) || x == INFINITY) bad_val = true;
+        t[i] = x * invT;
+      }
       if (d < 0 || d >= V) { bad_id = true; d = INT_MAX; }
-      t[i] = x * invT;
       id[i] = d;
       s_ids[warp][k] = d;
       m = fmaxf(m, t[i]);
@@ -263,28 +271,32 @@ __global__ void __launch_bounds__(ROW_WARPS * 32)
   m = warp_max(m);
   bad_val = __any_sync(0xffffffffu, bad_val);
   bad_id = __any_sync(0xffffffffu, bad_id);
+  float p[K_MAX / 32];
+  if (probs) {
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < K_MAX / 32; ++i) s += t[i];
+    s = warp_sum(s);
+    if (!(s > 0.f)) bad_val = true;
+    const float inv = s > 0.f ? 1.f / s : 0.f;
+#pragma unroll
+    for (int i = 0; i < K_MAX / 32; ++i) p[i] = t[i] * inv;
+  } else {
+    if (!(m > -INFINITY)) bad_val = true;
+    const float ms = (m > -INFINITY && m < INFINITY) ? m : 0.f;
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < K_MAX / 32; ++i)
+      if (lane + 32 * i < K) s += expf(t[i] - ms);
+    s = warp_sum(s);
+    const float lse = s > 0.f ? ms + logf(s) : INFINITY;
+#pragma unroll
+    for (int i = 0; i < K_MAX / 32; ++i) p[i] = (lane + 32 * i < K) ? expf(t[i] - lse) : 0.f;
+  }
   if (keep && lane == 0) {
     if (bad_id) atomicOr(&ctl->err, kErrBadIndex);
-    if (bad_val || !(m > -INFINITY)) atomicOr(&ctl->err, kErrBadTeacher);
+    if (bad_val) atomicOr(&ctl->err, kErrBadTeacher);
   }
-  const float ms = (m > -INFINITY && m < INFINITY) ? m : 0.f;
-  float s = 0.f;
-#pragma unroll
-  for (int i = 0; i < K_MAX / 32; ++i)
-    if (lane + 32 * i < K) s += expf(t[i] - ms);
-  s = warp_sum(s);
-  const float lse = s > 0.f ? ms + logf(s) : INFINITY;
-  float p[K_MAX / 32];
-  float pl = 0.f;
-#pragma unroll
-  for (int i = 0; i < K_MAX / 32; ++i) {
-    p[i] = 0.f;
-    if (lane + 32 * i < K) {
-      p[i] = expf(t[i] - lse);
-      if (p[i] > 0.f) pl += p[i] * (t[i] - lse);
-    }
-  }
-  pl = warp_sum(pl);
   __syncwarp();
 #pragma unroll
   for (int i = 0; i < K_MAX / 32; ++i) {
@@ -299,9 +311,20 @@ __global__ void __launch_bounds__(ROW_WARPS * 32)
       sp[(size_t)row * K + rk] = p[i];
       zs[(size_t)row * K + rk] = 0.f;
       s_sorted[warp][rk] = id[i];
+      s_sp[warp][rk] = p[i];
     }
   }
   __syncwarp();
+  // sum over distinct ids of P log P, P = the summed probability of an id
+  float pl = 0.f;
+  for (int j = lane; j < K; j += 32) {
+    const int idj = s_sorted[warp][j];
+    if (j > 0 && s_sorted[warp][j - 1] == idj) continue;  // not the first entry of its id
+    float P = 0.f;
+    for (int k = j; k < K && s_sorted[warp][k] == idj; ++k) P += s_sp[warp][k];
+    if (P > 0.f) pl += P * logf(P);
+  }
+  pl = warp_sum(pl);
   for (int vt = lane; vt <= NT; vt += 32) {  // lower bound of vt * 256 in the sorted ids
     const long long key = (long long)vt * BN;
     int lo = 0, hi = K;

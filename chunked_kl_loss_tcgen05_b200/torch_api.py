@@ -26,11 +26,11 @@ def _bits(t: torch.Tensor) -> torch.Tensor:
     raise TypeError(f"expected bfloat16 (or its uint16 bits), got {t.dtype}")
 
 
-def make_problem(hidden, W, topk_idx, T=1.0, chunk=0) -> FcklProblem:
+def make_problem(hidden, W, topk_idx, T=1.0, chunk=0, teacher=0) -> FcklProblem:
     N, H = hidden.shape
     V = W.shape[0]
     K = topk_idx.shape[1]
-    return FcklProblem(N, H, V, K, T, chunk)
+    return FcklProblem(N, H, V, K, T, chunk, teacher)
 
 
 def alloc_workspace(prob: FcklProblem, device) -> torch.Tensor:
@@ -52,13 +52,13 @@ def _check_inputs(hidden, W, topk_idx, topk_logit, row_mask):
 
 
 def fused_kl_fwd_bwd(hidden, W, topk_idx, topk_logit, row_mask=None, T=1.0, chunk=0,
-                     workspace=None, want_row_loss=False, check=True, out=None):
+                     workspace=None, want_row_loss=False, check=True, out=None, teacher=0):
     """Returns (loss[1], row_loss[N] or None, dH[N,H] fp32, dW[V,H] fp32).
 
     ``out``: optional (loss, dH, dW) tensors to write into instead of allocating."""
     hidden, W = _bits(hidden), _bits(W)
     _check_inputs(hidden, W, topk_idx, topk_logit, row_mask)
-    prob = make_problem(hidden, W, topk_idx, T, chunk)
+    prob = make_problem(hidden, W, topk_idx, T, chunk, teacher)
     dev = hidden.device
     if workspace is None:
         workspace = alloc_workspace(prob, dev)
@@ -89,11 +89,11 @@ def fused_kl_fwd_bwd(hidden, W, topk_idx, topk_logit, row_mask=None, T=1.0, chun
 
 
 def fused_kl_fwd(hidden, W, topk_idx, topk_logit, row_mask=None, T=1.0, chunk=0,
-                 workspace=None, want_row_loss=False, check=True):
+                 workspace=None, want_row_loss=False, check=True, teacher=0):
     """Returns (loss[1], row_loss[N] or None)."""
     hidden, W = _bits(hidden), _bits(W)
     _check_inputs(hidden, W, topk_idx, topk_logit, row_mask)
-    prob = make_problem(hidden, W, topk_idx, T, chunk)
+    prob = make_problem(hidden, W, topk_idx, T, chunk, teacher)
     dev = hidden.device
     if workspace is None:
         workspace = alloc_workspace(prob, dev)
@@ -205,12 +205,12 @@ def select_top_rows(score, n_select, row_mask=None):
 
 
 def fused_kl_rows(hidden, W, topk_idx, topk_logit, rows, T=1.0, chunk=0, workspace=None,
-                  grads=True, want_row_loss=False, check=True):
+                  grads=True, want_row_loss=False, check=True, teacher=0):
     """Loss (and dH, dW) over the listed rows only.  Returns (loss, row_loss, dH, dW)."""
     from . import fckl_fwd_bwd_rows
     hidden, W = _bits(hidden), _bits(W)
     _check_inputs(hidden, W, topk_idx, topk_logit, None)
-    prob = make_problem(hidden, W, topk_idx, T, chunk)
+    prob = make_problem(hidden, W, topk_idx, T, chunk, teacher)
     dev = hidden.device
     if workspace is None:
         workspace = alloc_workspace(prob, dev)

@@ -7,8 +7,11 @@
  *   z_r   = W h_r                         student logits over the vocabulary V
  *   q     = softmax(z_r / T)              over all V
  *   p     = softmax(topk_logit[r,:] / T)  over the K cached teacher ids, zero
- *                                         elsewhere
- *   l_r   = sum_k p_k (log p_k - log q[topk_idx[r,k]])     forward KL(p || q)
+ *                                         elsewhere (or given weights, see
+ *                                         fckl_teacher_format)
+ *   p~_v  = sum_{k: topk_idx[r,k] = v} p_k the dense teacher over V
+ *   l_r   = sum_v p~_v (log p~_v - log q_v)  forward KL(p~ || q); with distinct
+ *                                         ids = sum_k p_k (log p_k - log q[id_k])
  *   loss  = (1/N_v) sum_{valid r} l_r                      (0 when N_v = 0)
  *   dH_r  = dlogits_r W,  dW = sum_r dlogits_r^T h_r,
  *   dlogits_r = (q - p~) / (T N_v),  p~_v = sum_{k: topk_idx[r,k] = v} p_k,
@@ -86,13 +89,27 @@ typedef enum {
  * group's bf16 dlogits.  Live device bytes are O(max(chunk, 2048) * V) for the
  * workspace plus the caller's O(V * H) weights and gradients. */
 typedef struct {
-  int64_t N;      /* rows (batch * sequence)      */
-  int64_t H;      /* hidden size                  */
-  int64_t V;      /* vocabulary size              */
-  int32_t K;      /* cached teacher ids per row   */
-  float T;        /* temperature (> 0)            */
-  int64_t chunk;  /* rows per chunk, 0 = auto     */
+  int64_t N;        /* rows (batch * sequence)                  */
+  int64_t H;        /* hidden size                              */
+  int64_t V;        /* vocabulary size                          */
+  int32_t K;        /* cached teacher entries per row           */
+  float T;          /* temperature (> 0)                        */
+  int64_t chunk;    /* rows per chunk, 0 = auto                 */
+  int32_t teacher;  /* fckl_teacher_format of topk_logit        */
 } fckl_problem;
+
+/* What the teacher cache holds in topk_logit [N, K]:
+ *   FCKL_TEACHER_LOGITS  the top-K teacher logits; p = softmax(topk_logit / T)
+ *                        over the row's K entries ("offline top-K logits 방식").
+ *   FCKL_TEACHER_PROBS   non-negative class weights of sampled sparse targets
+ *                        (RS-KD, "기술 요약: 선택적 지식 증류의 재고", 방법론);
+ *                        p = topk_logit / sum(topk_logit) over the row, and T
+ *                        applies to the student only.  A valid row whose
+ *                        weights are negative, not finite or all zero is
+ *                        reported as FCKL_ERR_BAD_TEACHER.
+ * In both formats entries with the same id add into one class of the teacher
+ * distribution p~ (the dense teacher grid), so ids may repeat. */
+typedef enum { FCKL_TEACHER_LOGITS = 0, FCKL_TEACHER_PROBS = 1 } fckl_teacher_format;
 
 /* Bytes of device workspace fckl_fwd / fckl_fwd_bwd / fckl_fwd_bwd_rows /
  * fckl_student_entropy need for `prob` (0 when the problem is invalid): the

@@ -39,7 +39,12 @@ Readings taken where the pages are silent:
   * the reduction is the mean over valid rows of the flattened batch;
   * N_v = 0 gives L = 0 and zero gradients;
   * a teacher logit of -inf is allowed and gives p_k = 0 with 0 * log 0 := 0;
-  * repeated ids in one row are summed entry-wise into p~.
+  * repeated ids in one row add into one cell of the dense teacher p~ (the
+    dense-KL baseline expands the cache into the dense teacher grid), so the
+    loss is KL(p~ || q) over the distinct ids;
+  * teacher format "probs" (random-sampled sparse targets, "기술 요약: 선택적 지식
+    증류의 재고", section 방법론, RS-KD): the cache holds non-negative class
+    weights, p = w / sum(w), and the temperature applies to the student only.
 
 The oracle materialises each block's full [rows, V] fp64 softmax (the dense
 formulation); blocking over rows only regroups independent rows.
@@ -70,14 +75,22 @@ def log_softmax(x: np.ndarray, axis: int = -1) -> np.ndarray:
     return x - lse
 
 
-def teacher_distribution(topk_logit: np.ndarray, T: float):
-    """Softened teacher over the K cached ids: p = softmax(topk_logit / T).
+def teacher_distribution(topk_logit: np.ndarray, T: float, teacher: str = "logits"):
+    """Teacher probabilities over the K cache entries of each row.
 
-    aibase.it write-up, section "offline top-K logits 방식" (only the top-K
-    logits per position are kept); LLM Primer ch.6, section 6.2 (temperature).
-    Returns (p, log p), both [rows, K] float64."""
-    t = np.asarray(topk_logit, dtype=np.float64) / float(T)
-    logp = log_softmax(t, axis=1)
+    "logits": p = softmax(topk_logit / T) -- aibase.it write-up, section
+    "offline top-K logits 방식" (only the top-K logits per position are kept);
+    LLM Primer ch.6, section 6.2 (temperature).
+    "probs": p = w / sum(w) with w = topk_logit >= 0 -- sampled sparse targets
+    (RS-KD, "기술 요약: 선택적 지식 증류의 재고", section 방법론).
+    Returns (p, log p), both [rows, K] float64 (log p = -inf where p = 0)."""
+    x = np.asarray(topk_logit, dtype=np.float64)
+    if teacher == "probs":
+        tot = x.sum(axis=1, keepdims=True)
+        p = x / tot
+        with np.errstate(divide="ignore"):
+            return p, np.log(p)
+    logp = log_softmax(x / float(T), axis=1)
     return np.exp(logp), logp
 
 
@@ -100,13 +113,15 @@ def dense_teacher(p: np.ndarray, ids: np.ndarray, V: int) -> np.ndarray:
 def fused_chunked_kl(hidden: np.ndarray, W: np.ndarray, topk_idx: np.ndarray,
                      topk_logit: np.ndarray, row_mask: np.ndarray | None, T: float,
                      *, rows: np.ndarray | None = None, row_block: int = 256,
-                     grads: bool = True, return_dlogits: bool = False) -> dict:
+                     grads: bool = True, return_dlogits: bool = False,
+                     teacher: str = "logits") -> dict:
     """Loss and gradients of the fused chunked forward KL, in fp64.
 
     hidden [N, H] and W [V, H]: float arrays, or uint16 bf16 bit patterns
     (widened exactly; hidden one block of rows at a time).  topk_idx int
     [N, K] in [0, V), topk_logit [N, K], row_mask [N] (nonzero = row included;
-    None = all rows), temperature T > 0.
+    None = all rows), temperature T > 0, teacher format "logits" or "probs"
+    (see teacher_distribution).
 
     ``rows``: optional subset of rows to evaluate (masked ones are dropped;
     N_v still counts every valid row of the mask).  Without it every valid row
@@ -148,14 +163,14 @@ def fused_chunked_kl(hidden: np.ndarray, W: np.ndarray, topk_idx: np.ndarray,
             Hb = widen_bf16(hidden[rb]) if hidden_bits else np.asarray(hidden[rb], dtype=np.float64)
             Z = Hb @ W.T                                  # student logits [b, V]
             logq = student_log_probs(Z, T)                # normalised over all V
-            p, logp = teacher_distribution(topk_logit[rb], T)
+            p, logp = teacher_distribution(topk_logit[rb], T, teacher)
             ids = np.asarray(topk_idx[rb], dtype=np.int64)
-            logq_at = np.take_along_axis(logq, ids, axis=1)
-            with np.errstate(invalid="ignore"):
-                terms = np.where(p > 0.0, p * (logp - logq_at), 0.0)
+            P = dense_teacher(p, ids, V)            # [b, V]: repeated ids add up
+            with np.errstate(divide="ignore", invalid="ignore"):
+                terms = np.where(P > 0.0, P * (np.log(P) - logq), 0.0)
             out["row_loss_rows"][sel] = terms.sum(axis=1)
             if grads or return_dlogits:
-                G = (np.exp(logq) - dense_teacher(p, ids, V)) * grad_scale
+                G = (np.exp(logq) - P) * grad_scale
                 if return_dlogits:
                     out["dlogits_rows"][sel] = G
                 if grads:
@@ -173,7 +188,9 @@ def fused_chunked_kl(hidden: np.ndarray, W: np.ndarray, topk_idx: np.ndarray,
     return out
 
 
-def oracle_from_inputs(inp, *, rows=None, row_block: int = 256, grads: bool = True) -> dict:
+def oracle_from_inputs(inp, *, rows=None, row_block: int = 256, grads: bool = True,
+                       teacher: str = "logits") -> dict:
     """Run ``fused_chunked_kl`` on a ``synth.Inputs`` bundle (bf16 widened exactly)."""
     return fused_chunked_kl(inp.hidden, inp.W, inp.topk_idx, inp.topk_logit, inp.row_mask,
-                            inp.cfg.T, rows=rows, row_block=row_block, grads=grads)
+                            inp.cfg.T, rows=rows, row_block=row_block, grads=grads,
+                            teacher=teacher)

@@ -33,7 +33,7 @@ from __future__ import annotations
 import dataclasses
 import numpy as np
 
-__all__ = ["Config", "CONFIGS", "Inputs", "make_inputs", "make_custom",
+__all__ = ["Config", "CONFIGS", "Inputs", "make_inputs", "make_custom", "make_sampled_targets",
            "f32_to_bf16_bits", "bf16_bits_to_f32", "sample_rows"]
 
 _BLOCK_ELEMS = 1 << 24
@@ -157,3 +157,29 @@ def sample_rows(inp: Inputs, n: int = 64) -> np.ndarray:
     valid = np.nonzero(inp.row_mask)[0]
     n = min(n, valid.size)
     return np.sort(r_s.choice(valid, size=n, replace=False)).astype(np.int64)
+
+
+def make_sampled_targets(N: int, H: int, V: int, K: int, T: float = 1.0, sigma: float = 3.0,
+                         mask_frac: float = 0.0, seed: int = 0, chunk: int = 0) -> Inputs:
+    """Sparse sampled teacher targets (RS-KD form): per row a synthetic teacher
+    over a candidate set of min(4K, V) distinct ids with logits N(0, sigma),
+    K ids drawn WITH replacement from it, and one positive weight per draw
+    (uniform in [0.5, 1.5)); ``topk_logit`` holds those weights.  hidden, W and
+    the mask follow the usual recipe (streams 0, 1, 4); stream 2 draws the
+    candidates and samples, stream 3 the candidate logits and the weights."""
+    base = make_custom(N, H, V, 1, T=T, sigma=sigma, mask_frac=mask_frac, seed=seed, chunk=chunk,
+                       name="sampled_targets")
+    ss = np.random.SeedSequence(seed)
+    _, _, r_id, r_lg, _, _ = [np.random.Generator(np.random.PCG64(x)) for x in ss.spawn(6)]
+    C = min(4 * K, V)
+    ids = np.empty((N, K), np.int32)
+    w = np.empty((N, K), np.float32)
+    for r in range(N):
+        cand = r_id.choice(V, size=C, replace=False)
+        lg = r_lg.standard_normal(C) * sigma
+        pr = np.exp(lg - lg.max())
+        pr /= pr.sum()
+        ids[r] = cand[r_id.choice(C, size=K, replace=True, p=pr)]
+        w[r] = r_lg.uniform(0.5, 1.5, K).astype(np.float32)
+    cfg = dataclasses.replace(base.cfg, K=K)
+    return Inputs(cfg, base.hidden, base.W, ids, w, base.row_mask)

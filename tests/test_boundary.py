@@ -66,7 +66,7 @@ def test_workspace_and_chunk_rules():
 
 @pytest.mark.parametrize("bad", [
     dict(N=0), dict(H=0), dict(V=0), dict(K=0), dict(T=0.0), dict(T=-1.0),
-    dict(T=float("nan")), dict(T=float("inf")), dict(chunk=-1)])
+    dict(T=float("nan")), dict(T=float("inf")), dict(chunk=-1), dict(teacher=2), dict(teacher=-1)])
 def test_invalid_problem_rejected(bad):
     kw = dict(N=64, H=64, V=512, K=8, T=1.0, chunk=0)
     kw.update(bad)

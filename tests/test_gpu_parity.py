@@ -195,3 +195,47 @@ def test_teacher_row_without_finite_logit_is_reported():
     lg = inp.topk_logit.copy()
     lg[3, 2] = np.nan
     assert _raw_call(inp, logits=lg) == FCKL_ERR_BAD_TEACHER
+
+
+# ------------------------------------------------ sampled sparse targets (RS-KD)
+@pytest.mark.parametrize("shape", [(300, 128, 2000, 24, 1.0, 128), (517, 64, 777, 64, 2.0, 0),
+                                   (256, 256, 4096, 100, 1.0, 64)])
+def test_sampled_target_teacher_full(shape):
+    """Teacher given as sampled class weights (repeats allowed): p = w / sum w."""
+    N, H, V, K, T, chunk = shape
+    inp = synth.make_sampled_targets(N, H, V, K, T=T, mask_frac=0.1, seed=61 + N, chunk=chunk)
+    s = np.sort(inp.topk_idx, axis=1)
+    assert (s[:, 1:] == s[:, :-1]).any()          # the draws do repeat ids
+    d = arrays_to_device(inp.hidden, inp.W, inp.topk_idx, inp.topk_logit, inp.row_mask)
+    loss, rl, dH, dW = fused_kl_fwd_bwd(*d, T=T, chunk=chunk, want_row_loss=True, teacher=1)
+    torch.cuda.synchronize()
+    o = oracle.oracle_from_inputs(inp, teacher="probs")
+    check_full(inp, dict(loss=loss.item(), row_loss=rl.cpu().numpy(), dH=dH, dW=dW), o)
+
+
+def test_repeated_ids_in_logit_cache():
+    """Repeated ids in a top-K logit cache add into one teacher class."""
+    inp = synth.make_custom(300, 128, 2000, 10, mask_frac=0.1, seed=71, chunk=128)
+    inp.topk_idx[::3, 4] = inp.topk_idx[::3, 1]
+    inp.topk_idx[::5, 9] = inp.topk_idx[::5, 2]
+    o = oracle.oracle_from_inputs(inp)
+    check_full(inp, run_gpu(inp), o)
+
+
+def test_bad_sampled_weights_are_reported():
+    inp = synth.make_sampled_targets(64, 64, 512, 8, seed=72)
+    d = list(arrays_to_device(inp.hidden, inp.W, inp.topk_idx, inp.topk_logit, None))
+    from chunked_kl_loss_tcgen05_b200 import FcklError
+    for bad in (-0.5, float("nan"), float("inf")):
+        lg = inp.topk_logit.copy()
+        lg[7, 3] = bad
+        d[3] = torch.from_numpy(lg).cuda()
+        with pytest.raises(FcklError) as ei:
+            fused_kl_fwd_bwd(*d, teacher=1)
+        assert ei.value.status == FCKL_ERR_BAD_TEACHER
+    lg = inp.topk_logit.copy()
+    lg[5, :] = 0.0                                 # a row with no mass
+    d[3] = torch.from_numpy(lg).cuda()
+    with pytest.raises(FcklError) as ei:
+        fused_kl_fwd_bwd(*d, teacher=1)
+    assert ei.value.status == FCKL_ERR_BAD_TEACHER

@@ -243,20 +243,59 @@ def test_no_valid_rows():
     assert not o["dH"].any() and not o["dW"].any()
 
 
-def test_duplicate_ids_sum_entrywise():
-    """Repeated ids: the loss is the entry-wise sum and p~ adds both entries;
-    checked against autograd of the entry-wise gather formulation."""
+def test_duplicate_ids_add_into_one_dense_cell():
+    """Repeated ids: the teacher is the dense grid p~ (entries of one id add up)
+    and the loss is KL(p~ || q); checked against scipy's KL of the dense grid and
+    autograd of kl_div on it."""
     h, W, ids, lg, mask, T = _rand_case(82, K=5)
     ids[:, 3] = ids[:, 1]
     o = oracle.fused_chunked_kl(h, W, ids, lg, mask, T)
+    q = scipy.special.softmax((h @ W.T) / T, axis=1)
+    pk = scipy.special.softmax(lg / T, axis=1)
+    for r in range(h.shape[0]):
+        pd = np.zeros(W.shape[0])
+        np.add.at(pd, ids[r], pk[r])
+        np.testing.assert_allclose(o["row_loss"][r], scipy.stats.entropy(pd, q[r]), rtol=1e-11)
     th = torch.tensor(h, requires_grad=True); tW = torch.tensor(W, requires_grad=True)
     logq = F.log_softmax(th @ tW.T / T, dim=1)
-    logp = F.log_softmax(torch.tensor(lg) / T, dim=1)
-    g = torch.gather(logq, 1, torch.tensor(ids.astype(np.int64)))
-    loss = (logp.exp() * (logp - g)).sum() / h.shape[0]
+    pd = torch.zeros(h.shape[0], W.shape[0], dtype=torch.float64)
+    pd.scatter_add_(1, torch.tensor(ids.astype(np.int64)), torch.softmax(torch.tensor(lg) / T, 1))
+    loss = F.kl_div(logq, pd, reduction="sum") / h.shape[0]
     loss.backward()
     np.testing.assert_allclose(o["loss"], loss.item(), rtol=1e-12)
     np.testing.assert_allclose(o["dW"], tW.grad.numpy(), rtol=1e-9, atol=1e-15)
+
+
+def test_probs_teacher_matches_scipy_and_autograd():
+    """Teacher given as sampled class weights (RS-KD): p = w / sum(w), repeats
+    allowed (sampling with replacement), temperature on the student only."""
+    rng = np.random.default_rng(90)
+    h, W, _, _, mask, _ = _rand_case(91, N=10, V=40, mask_frac=0.2)
+    K, T = 12, 1.7
+    ids = rng.integers(0, 40, (10, K)).astype(np.int32)          # repeats are likely
+    w = rng.random((10, K)) * (rng.random((10, K)) < 0.8)        # some zero weights
+    w[:, 0] += 0.1
+    o = oracle.fused_chunked_kl(h, W, ids, w, mask, T, teacher="probs")
+    q = scipy.special.softmax((h @ W.T) / T, axis=1)
+    for r in range(10):
+        if not mask[r]:
+            continue
+        pd = np.zeros(40)
+        np.add.at(pd, ids[r], w[r] / w[r].sum())
+        np.testing.assert_allclose(o["row_loss"][r], scipy.stats.entropy(pd, q[r]), rtol=1e-11)
+    th = torch.tensor(h, requires_grad=True); tW = torch.tensor(W, requires_grad=True)
+    logq = F.log_softmax(th @ tW.T / T, dim=1)
+    pd = torch.zeros(10, 40, dtype=torch.float64)
+    pd.scatter_add_(1, torch.tensor(ids.astype(np.int64)), torch.tensor(w / w.sum(1, keepdims=True)))
+    keep = torch.tensor(mask != 0)
+    loss = F.kl_div(logq[keep], pd[keep], reduction="sum") / keep.sum()
+    loss.backward()
+    np.testing.assert_allclose(o["loss"], loss.item(), rtol=1e-12)
+    np.testing.assert_allclose(o["dH"], th.grad.numpy(), rtol=1e-9, atol=1e-15)
+    np.testing.assert_allclose(o["dW"], tW.grad.numpy(), rtol=1e-9, atol=1e-15)
+    # scaling the weights of a row changes nothing
+    o2 = oracle.fused_chunked_kl(h, W, ids, w * 3.5, mask, T, teacher="probs")
+    np.testing.assert_allclose(o2["row_loss"], o["row_loss"], rtol=1e-12)
 
 
 def test_row_subset_matches_full():
@@ -291,7 +330,7 @@ def _mutant(kind):
             if kind == "student_no_T":
                 okl.student_log_probs = lambda Z, T_: saved[0](Z, 1.0)
             elif kind == "teacher_no_T":
-                okl.teacher_distribution = lambda lg_, T_: saved[1](lg_, 1.0)
+                okl.teacher_distribution = lambda lg_, T_, *a: saved[1](lg_, 1.0, *a)
             elif kind == "q_over_topk_only":
                 # normalising the student only over a prefix of the vocabulary
                 okl.student_log_probs = lambda Z, T_: okl.log_softmax(
@@ -301,8 +340,8 @@ def _mutant(kind):
             elif kind == "id_off_by_one":
                 ids = (ids + 1) % W.shape[0]
             elif kind == "reverse_kl_weights":
-                okl.teacher_distribution = lambda lg_, T_: (
-                    lambda pl: (np.full_like(pl[0], 1.0 / pl[0].shape[1]), pl[1]))(saved[1](lg_, T_))
+                okl.teacher_distribution = lambda lg_, T_, *a: (
+                    lambda pl: (np.full_like(pl[0], 1.0 / pl[0].shape[1]), pl[1]))(saved[1](lg_, T_, *a))
             return okl.fused_chunked_kl(h, W, ids, lg, mask, T, **kw)
         finally:
             okl.student_log_probs, okl.teacher_distribution, okl.dense_teacher = saved
