@@ -84,27 +84,26 @@ struct EpiLseT {
           nid = cur < p.K ? __ldg(rid + cur) : INT_MAX;
         }
       }
-      float cm = -INFINITY;
+      // Max over the raw logits first (scale2 > 0 keeps the order), then one
+      // FMA per element forms a - max inside the exp2.
       const bool full = base + 32 <= p.V;
-      if (full) {
+      if (!full) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) { v[j] *= p.scale2; cm = fmaxf(cm, v[j]); }
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          v[j] = (base + j < p.V) ? v[j] * p.scale2 : -INFINITY;
-          cm = fmaxf(cm, v[j]);
-        }
+        for (int j = 0; j < 32; ++j) v[j] = (base + j < p.V) ? v[j] : -INFINITY;
       }
-      if (cm == -INFINITY) continue;
-      const float nm = fmaxf(m, cm);
-      const float rescale = exp2f(m - nm);
+      float cz = v[0];
+#pragma unroll
+      for (int j = 1; j < 32; ++j) cz = fmaxf(cz, v[j]);
+      if (cz == -INFINITY) continue;
+      const float nm = fmaxf(m, cz * p.scale2);
+      const float rescale = ex2_approx(m - nm);
       float acc = 0.f, uacc = 0.f;
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        const float e = exp2f(v[j] - nm);
+        const float a = v[j] * p.scale2;
+        const float e = ex2_approx(fmaf(v[j], p.scale2, -nm));
         acc += e;
-        if (kEntropy) uacc += (full || e > 0.f) ? e * v[j] : 0.f;
+        if (kEntropy) uacc += (full || e > 0.f) ? e * a : 0.f;
       }
       s = s * rescale + acc;
       if (kEntropy) u = u * rescale + uacc;
@@ -172,10 +171,11 @@ struct EpiDlogits {
     }
     if (base + 32 <= p.V) {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = exp2f(fmaf(v[j], p.scale2, -lse));
+      for (int j = 0; j < 32; ++j) v[j] = ex2_approx(fmaf(v[j], p.scale2, -lse));
     } else {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = (base + j < p.V) ? exp2f(fmaf(v[j], p.scale2, -lse)) : 0.f;
+      for (int j = 0; j < 32; ++j)
+        v[j] = (base + j < p.V) ? ex2_approx(fmaf(v[j], p.scale2, -lse)) : 0.f;
     }
     while (st.nid < base + 32) {  // subtract the teacher mass at cached ids
       const int j = st.nid - base;

@@ -24,7 +24,7 @@ namespace {
 constexpr size_t kAlign = 256;
 constexpr int kMaxDevices = 64;
 
-constexpr long long kDwRows = 2048;  // minimum reduction depth of a dW launch (rows)
+constexpr long long kDwRows = 4096;  // minimum reduction depth of a dW launch (rows)
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }

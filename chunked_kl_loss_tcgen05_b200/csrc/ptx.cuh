@@ -161,6 +161,14 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
       : "memory");
 }
 
+// 2^x with the SFU's approximate exp2 instruction (flush-to-zero; relative
+// error about 2^-22, far inside what bf16 operands and fp32 sums need).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Shared-memory matrix descriptor for a 128-byte-swizzled tile (sm_100 format:
 // start >> 4 in bits 0-13, leading byte offset >> 4 in 16-29, stride byte
 // offset >> 4 in 32-45, version 1 in 46-47, swizzle mode 2 (128B) in 61-63).

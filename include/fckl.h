@@ -84,9 +84,9 @@ typedef enum {
 /* Problem description.  chunk = rows per chunk (0 = automatic: the largest
  * multiple of 128 rows whose bf16 dlogits block [chunk, V] fits in 512 MiB,
  * capped at N rounded up to 64).  The dW GEMM runs once per group of
- * ceil(2048 / chunk) consecutive chunks (at most all of them), so that each
- * read-modify-write of dW covers at least 2048 rows; the workspace holds that
- * group's bf16 dlogits.  Live device bytes are O(max(chunk, 2048) * V) for the
+ * ceil(4096 / chunk) consecutive chunks (at most all of them), so that each
+ * read-modify-write of dW covers at least 4096 rows; the workspace holds that
+ * group's bf16 dlogits.  Live device bytes are O(max(chunk, 4096) * V) for the
  * workspace plus the caller's O(V * H) weights and gradients. */
 typedef struct {
   int64_t N;        /* rows (batch * sequence)                  */

@@ -60,8 +60,8 @@ def test_workspace_and_chunk_rules():
     a = fk.fckl_workspace_bytes(FcklProblem(32768, 4096, 128256, 100, 1.0, 1024))
     b = fk.fckl_workspace_bytes(FcklProblem(65536, 4096, 128256, 100, 1.0, 1024))
     assert b - a == 32768 * 4                           # only the per-row loss grows
-    # chunk 1024 < 2048: two chunks of dlogits feed one dW GEMM
-    assert 2 * 1024 * 128256 * 2 <= a < 560 * 2**20
+    # chunk 1024 < 4096: four chunks of dlogits feed one dW GEMM
+    assert 4 * 1024 * 128256 * 2 <= a < 1100 * 2**20
 
 
 @pytest.mark.parametrize("bad", [
