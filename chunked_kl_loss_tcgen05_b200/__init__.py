@@ -50,10 +50,11 @@ class FcklProblem(ctypes.Structure):
     """Mirror of ``fckl_problem``."""
     _fields_ = [("N", ctypes.c_int64), ("H", ctypes.c_int64), ("V", ctypes.c_int64),
                 ("K", ctypes.c_int32), ("T", ctypes.c_float), ("chunk", ctypes.c_int64),
-                ("teacher", ctypes.c_int32)]
+                ("teacher", ctypes.c_int32), ("n_valid_total", ctypes.c_int64)]
 
-    def __init__(self, N, H, V, K, T=1.0, chunk=0, teacher=FCKL_TEACHER_LOGITS):
-        super().__init__(int(N), int(H), int(V), int(K), float(T), int(chunk), int(teacher))
+    def __init__(self, N, H, V, K, T=1.0, chunk=0, teacher=FCKL_TEACHER_LOGITS, n_valid_total=0):
+        super().__init__(int(N), int(H), int(V), int(K), float(T), int(chunk), int(teacher),
+                         int(n_valid_total))
 
 
 class FcklKernelStat(ctypes.Structure):

@@ -43,6 +43,7 @@ bool valid_problem(const fckl_problem* p) {
   if (!(std::isfinite(p->T) && p->T > 0.f)) return false;
   if (p->N > INT32_MAX || p->H > INT32_MAX || p->V > INT32_MAX) return false;
   if (p->teacher != FCKL_TEACHER_LOGITS && p->teacher != FCKL_TEACHER_PROBS) return false;
+  if (p->n_valid_total < 0 || p->n_valid_total > INT32_MAX) return false;
   return true;
 }
 
@@ -334,10 +335,11 @@ fckl_status run(const Request& q) {
   if (cudaMemsetAsync(ctl, 0, sizeof(DeviceCtl), st) != cudaSuccess) return FCKL_ERR_CUDA;
   if (!ent) {
     ProfScope ps(K_COUNT, st, 0.0, list ? q.n_rows * 4.0 : (q.row_mask ? (double)L.N : 0.0));
+    const int nv_total = (int)prob->n_valid_total;
     if (list)
-      k_count_list<<<1, 1024, 0, st>>>(q.rows, q.n_rows, L.N, ctl);
+      k_count_list<<<1, 1024, 0, st>>>(q.rows, q.n_rows, L.N, nv_total, ctl);
     else
-      k_count_valid<<<1, 1024, 0, st>>>(q.row_mask, L.N, ctl);
+      k_count_valid<<<1, 1024, 0, st>>>(q.row_mask, L.N, nv_total, ctl);
   }
   if (list) {  // rows that are not listed get zero row loss and zero dH
     if (cudaMemsetAsync(rl, 0, (size_t)L.N * 4, st) != cudaSuccess) return FCKL_ERR_CUDA;

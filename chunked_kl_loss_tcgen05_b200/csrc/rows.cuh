@@ -24,9 +24,10 @@ __device__ __forceinline__ float warp_sum(float x) {
   return x;
 }
 
-// N_valid = #rows with row_mask != 0 (N when there is no mask).  One block.
+// N_valid = #rows with row_mask != 0 (N when there is no mask), or the
+// caller's total (> 0) when the rows are one shard of a larger batch.  One block.
 __global__ void __launch_bounds__(1024) k_count_valid(const uint8_t* __restrict__ mask, long long N,
-                                                      DeviceCtl* ctl) {
+                                                      int total, DeviceCtl* ctl) {
   __shared__ int red[32];
   int c = 0;
   if (mask == nullptr) {
@@ -42,14 +43,14 @@ __global__ void __launch_bounds__(1024) k_count_valid(const uint8_t* __restrict_
     c = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
-    if (threadIdx.x == 0) ctl->n_valid = c;
+    if (threadIdx.x == 0) ctl->n_valid = total > 0 ? total : c;
   }
 }
 
 // N_valid for a row list: entries in [0, N) count; negative entries are
 // padding and are skipped; entries >= N are reported as bad indices.  One block.
 __global__ void __launch_bounds__(1024) k_count_list(const int32_t* __restrict__ rows, long long n,
-                                                     long long N, DeviceCtl* ctl) {
+                                                     long long N, int total, DeviceCtl* ctl) {
   __shared__ int red[32];
   int c = 0;
   bool bad = false;
@@ -67,7 +68,7 @@ __global__ void __launch_bounds__(1024) k_count_list(const int32_t* __restrict__
     c = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
-    if (threadIdx.x == 0) ctl->n_valid = c;
+    if (threadIdx.x == 0) ctl->n_valid = total > 0 ? total : c;
   }
 }
 

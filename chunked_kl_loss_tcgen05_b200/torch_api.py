@@ -26,11 +26,11 @@ def _bits(t: torch.Tensor) -> torch.Tensor:
     raise TypeError(f"expected bfloat16 (or its uint16 bits), got {t.dtype}")
 
 
-def make_problem(hidden, W, topk_idx, T=1.0, chunk=0, teacher=0) -> FcklProblem:
+def make_problem(hidden, W, topk_idx, T=1.0, chunk=0, teacher=0, n_valid_total=0) -> FcklProblem:
     N, H = hidden.shape
     V = W.shape[0]
     K = topk_idx.shape[1]
-    return FcklProblem(N, H, V, K, T, chunk, teacher)
+    return FcklProblem(N, H, V, K, T, chunk, teacher, n_valid_total)
 
 
 def alloc_workspace(prob: FcklProblem, device) -> torch.Tensor:
@@ -52,13 +52,16 @@ def _check_inputs(hidden, W, topk_idx, topk_logit, row_mask):
 
 
 def fused_kl_fwd_bwd(hidden, W, topk_idx, topk_logit, row_mask=None, T=1.0, chunk=0,
-                     workspace=None, want_row_loss=False, check=True, out=None, teacher=0):
+                     workspace=None, want_row_loss=False, check=True, out=None, teacher=0,
+                     n_valid_total=0):
     """Returns (loss[1], row_loss[N] or None, dH[N,H] fp32, dW[V,H] fp32).
 
-    ``out``: optional (loss, dH, dW) tensors to write into instead of allocating."""
+    ``out``: optional (loss, dH, dW) tensors to write into instead of allocating.
+    ``n_valid_total``: N_v for the mean and gradient scale when these rows are one
+    shard of a larger batch (0 = the valid rows of this call)."""
     hidden, W = _bits(hidden), _bits(W)
     _check_inputs(hidden, W, topk_idx, topk_logit, row_mask)
-    prob = make_problem(hidden, W, topk_idx, T, chunk, teacher)
+    prob = make_problem(hidden, W, topk_idx, T, chunk, teacher, n_valid_total)
     dev = hidden.device
     if workspace is None:
         workspace = alloc_workspace(prob, dev)

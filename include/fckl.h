@@ -96,6 +96,10 @@ typedef struct {
   float T;          /* temperature (> 0)                        */
   int64_t chunk;    /* rows per chunk, 0 = auto                 */
   int32_t teacher;  /* fckl_teacher_format of topk_logit        */
+  int64_t n_valid_total; /* 0: N_v = the valid rows of this call;
+                            > 0: N_v used for the mean and the gradient
+                            scale, e.g. the valid rows of all data-parallel
+                            ranks, each rank passing its own row shard */
 } fckl_problem;
 
 /* What the teacher cache holds in topk_logit [N, K]:

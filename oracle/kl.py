@@ -114,14 +114,16 @@ def fused_chunked_kl(hidden: np.ndarray, W: np.ndarray, topk_idx: np.ndarray,
                      topk_logit: np.ndarray, row_mask: np.ndarray | None, T: float,
                      *, rows: np.ndarray | None = None, row_block: int = 256,
                      grads: bool = True, return_dlogits: bool = False,
-                     teacher: str = "logits") -> dict:
+                     teacher: str = "logits", n_valid: int | None = None) -> dict:
     """Loss and gradients of the fused chunked forward KL, in fp64.
 
     hidden [N, H] and W [V, H]: float arrays, or uint16 bf16 bit patterns
     (widened exactly; hidden one block of rows at a time).  topk_idx int
     [N, K] in [0, V), topk_logit [N, K], row_mask [N] (nonzero = row included;
     None = all rows), temperature T > 0, teacher format "logits" or "probs"
-    (see teacher_distribution).
+    (see teacher_distribution).  ``n_valid``: the N_v of the mean and of the
+    gradient scale when these rows are one shard of a larger batch (default:
+    the valid rows of ``row_mask``).
 
     ``rows``: optional subset of rows to evaluate (masked ones are dropped;
     N_v still counts every valid row of the mask).  Without it every valid row
@@ -141,7 +143,7 @@ def fused_chunked_kl(hidden: np.ndarray, W: np.ndarray, topk_idx: np.ndarray,
     N, H = hidden.shape
     V = W.shape[0]
     mask = np.ones(N, dtype=bool) if row_mask is None else (np.asarray(row_mask) != 0)
-    n_valid = int(mask.sum())
+    n_valid = int(mask.sum()) if n_valid is None else int(n_valid)
     if rows is None:
         todo = np.nonzero(mask)[0]
     else:

@@ -239,3 +239,43 @@ def test_bad_sampled_weights_are_reported():
     with pytest.raises(FcklError) as ei:
         fused_kl_fwd_bwd(*d, teacher=1)
     assert ei.value.status == FCKL_ERR_BAD_TEACHER
+
+
+def test_global_valid_count_scales_loss_and_grads():
+    """n_valid_total (the N_v of all data-parallel shards) replaces the local
+    count in the mean and the gradient scale: doubling it halves everything."""
+    inp = synth.make_custom(300, 128, 2000, 10, mask_frac=0.1, seed=81, chunk=128)
+    d = arrays_to_device(inp.hidden, inp.W, inp.topk_idx, inp.topk_logit, inp.row_mask)
+    l1, _, dH1, dW1 = fused_kl_fwd_bwd(*d, chunk=128)
+    nv = int((inp.row_mask != 0).sum())
+    l2, _, dH2, dW2 = fused_kl_fwd_bwd(*d, chunk=128, n_valid_total=2 * nv)
+    torch.cuda.synchronize()
+    assert l2.item() == pytest.approx(l1.item() / 2, rel=1e-6)
+    assert rel_fro(dH2.cpu().numpy(), dH1.cpu().numpy() / 2) < 1e-6
+    assert rel_fro(dW2.cpu().numpy(), dW1.cpu().numpy() / 2) < 1e-6
+    o = oracle.oracle_from_inputs(inp)
+    o2 = oracle.fused_chunked_kl(inp.hidden, inp.W, inp.topk_idx, inp.topk_logit, inp.row_mask,
+                                 inp.cfg.T, n_valid=2 * nv)
+    assert abs(l2.item() - o2["row_loss"].sum() / (2 * nv)) <= LOSS_RTOL * abs(o["loss"] / 2)
+
+
+def test_dp_wrapper_single_rank_nccl():
+    """The data-parallel wrapper on one NCCL rank equals the plain call."""
+    import torch.distributed as dist
+    from chunked_kl_loss_tcgen05_b200.dp import fused_kl_fwd_bwd_dp
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1)
+    try:
+        inp = synth.make_custom(300, 128, 2000, 10, mask_frac=0.1, seed=82, chunk=128)
+        d = arrays_to_device(inp.hidden, inp.W, inp.topk_idx, inp.topk_logit, inp.row_mask)
+        l1, _, dH1, dW1 = fused_kl_fwd_bwd(*d, chunk=128)
+        l2, dH2, dW2 = fused_kl_fwd_bwd_dp(*d, chunk=128)
+        torch.cuda.synchronize()
+        assert l2.item() == pytest.approx(l1.item(), rel=1e-6)
+        assert rel_fro(dW2.cpu().numpy(), dW1.cpu().numpy()) < 1e-6
+        assert rel_fro(dH2.cpu().numpy(), dH1.cpu().numpy()) < 1e-6
+    finally:
+        dist.destroy_process_group()
