@@ -34,6 +34,14 @@ METRIC = "fused KL fwd+bwd tokens/s & TFLOP/s (frac of BF16 peak); peak GiB vs s
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                   "source": "fallback"}
 
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum, mean over the
+# launches of one call) from the ncu capture of the current kernels on this workload,
+# summarised under profiles/.  Reset an entry to None when its kernel changes.
+MEASURED_TRAFFIC = {
+    "llama8b_to_3b_8k_N8192_H3072_V128256_K100": {
+        "fwd_logits_lse": 0.817e9, "bwd_dlogits": 1.327e9, "dH_gemm": 3.00e9, "dW_gemm": 3.77e9},
+}
+
 
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -276,14 +284,15 @@ def run_cuda(args):
             roofline = {"kernel": dom["name"], "bound": "tensor", "achieved": ach, "peak": peak,
                         "unit": "TFLOP/s", "frac": ach / peak,
                         "peak_kind": f"bf16_tflops_sustained ({peaks['source']})",
-                        "traffic": None,
+                        "traffic": MEASURED_TRAFFIC.get(cfg.name, {}).get(dom["name"]),
+                        "algorithmic_bytes": dom["bytes"] / dom["launches"],
                         "share": dom["total_ms"] / args.steps / ms_step}
         else:
             peak = peaks["hbm_gbs"]
             ach = dom["bytes"] / dom["launches"] / (avg_ms / 1e3) / 1e9
             roofline = {"kernel": dom["name"], "bound": "hbm", "achieved": ach, "peak": peak,
                         "unit": "GB/s", "frac": ach / peak, "peak_kind": f"hbm_gbs ({peaks['source']})",
-                        "traffic": None,
+                        "traffic": MEASURED_TRAFFIC.get(cfg.name, {}).get(dom["name"]),
                         "share": dom["total_ms"] / args.steps / ms_step}
     kernels = [{"name": p["name"], "launches": p["launches"], "ms_per_step": p["total_ms"] / 2,
                 "share": p["total_ms"] / bd_total,
