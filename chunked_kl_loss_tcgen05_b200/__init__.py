@@ -186,7 +186,7 @@ def fckl_status_string(status: int) -> str:
 
 KERNEL_KINDS = ("count_valid", "prep_teacher", "fwd_logits_lse", "merge_loss", "bwd_dlogits",
                 "dH_gemm", "dW_gemm", "finalize", "entropy_gemm", "merge_entropy", "gather_rows",
-                "scatter_rows", "select_rows")
+                "scatter_rows", "select_rows", "zero_dw")
 
 
 def fckl_profile_begin(kinds=None) -> None:

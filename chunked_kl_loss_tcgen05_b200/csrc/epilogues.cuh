@@ -45,7 +45,6 @@ struct EpiLseT {
   static constexpr uint32_t kSmemBytes = 0;
   static constexpr bool kUsesMapC = false;
   struct Params {
-    int rows_c;               // valid rows of this chunk
     int V, K, NT;
     float scale2;             // log2(e) / T
     const int* sid;           // [rows_c, K] ids sorted ascending (invalid ids -> INT_MAX)
@@ -59,7 +58,7 @@ struct EpiLseT {
   static __device__ void tile(const Params& p, State&, const Work& w, uint32_t taddr, int r,
                               const CUtensorMap*, int, int) {
     const int row = w.m0 + r;
-    const bool rv = row < p.rows_c;
+    const bool rv = row < w.rows;
     const int* rid = p.sid + (size_t)(rv ? row : 0) * p.K;
     int cur = 0, nid = INT_MAX;
     if (kGather && rv) {
@@ -143,9 +142,9 @@ __device__ __forceinline__ void stage_release() {
 
 struct EpiDlogits {
   static constexpr uint32_t kSmemBytes = 4 * 2 * 4096;
-  static constexpr bool kUsesMapC = true;  // map C: dlogits [rows_c, V] bf16, box {64, 32}
+  static constexpr bool kUsesMapC = true;  // map C: dlogits [rows, V] bf16, box {64, 32}
   struct Params {
-    int rows_c, V, K, NT;
+    int V, K, NT;
     float scale2;             // log2(e) / T
     const float* lse2;        // [rows_c] log2-domain log-sum-exp of z / T
     const int* sid;           // [rows_c, K] sorted ids
@@ -189,7 +188,7 @@ struct EpiDlogits {
   static __device__ void tile(const Params& p, State& st, const Work& w, uint32_t taddr, int r,
                               const CUtensorMap* mapC, int quarter, int lane) {
     const int row = w.m0 + r;
-    const bool rv = row < p.rows_c;
+    const bool rv = row < w.rows;
     const bool keep = rv && (p.mask == nullptr || p.mask[row] != 0);
     const int* rid = p.sid + (size_t)(rv ? row : 0) * p.K;
     const float* rp = p.sp + (size_t)(rv ? row : 0) * p.K;
@@ -225,7 +224,7 @@ struct EpiDlogits {
                                                     pack_bf16x2(v1[8 * j + 6], v1[8 * j + 7]));
       stage_release();
       if (lane == 0) {  // one group per slice, empty when the slice lies outside the map
-        if (base < p.V && y < p.rows_c) tma_store_2d(mapC, smem_u32(buf), base, y);
+        if (base < p.V && y < w.rows) tma_store_2d(mapC, smem_u32(buf), base, y);
         bulk_commit();
       }
       ++st.n;
@@ -269,9 +268,9 @@ __device__ __forceinline__ void stage_fp32_slices(uint8_t* bufs, int& n, uint32_
 
 struct EpiDH {
   static constexpr uint32_t kSmemBytes = 4 * 2 * 4096;
-  static constexpr bool kUsesMapC = true;  // map C: dH chunk rows [rows_c, H] fp32, box {32, 32}
+  static constexpr bool kUsesMapC = true;  // map C: dH chunk rows [rows, H] fp32, box {32, 32}
   struct Params {
-    int rows_c, H;
+    int H;
     float invT;
     const DeviceCtl* ctl;
   };
@@ -289,8 +288,7 @@ struct EpiDH {
   static __device__ void tile(const Params& p, State& st, const Work& w, uint32_t taddr, int,
                               const CUtensorMap* mapC, int quarter, int lane) {
     const int y = w.m0 + quarter * 32;
-    stage_fp32_slices<true>(st.buf, st.n, taddr, st.alpha, mapC, w.n0, p.H, y, y < p.rows_c,
-                            lane);
+    stage_fp32_slices<true>(st.buf, st.n, taddr, st.alpha, mapC, w.n0, p.H, y, y < w.rows, lane);
   }
   static __device__ void finish(const Params&, State&, int lane) {
     if (lane == 0) bulk_wait_all();

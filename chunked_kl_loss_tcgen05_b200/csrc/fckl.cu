@@ -34,7 +34,7 @@ struct Layout {
   long long G;  // chunks per dW group: dlogits of G chunks feed one dW GEMM
   size_t off_rowloss, off_sid, off_sp, off_zs, off_tstart, off_plogp, off_lse2, off_part,
       off_upart, off_hstage, off_idstage, off_lgstage, off_mstage, off_dhstage, off_rlstage,
-      off_dlog, total;
+      off_list, off_dlog, total;
 };
 
 bool valid_problem(const fckl_problem* p) {
@@ -95,6 +95,7 @@ Layout make_layout(const fckl_problem* p, bool full = true) {
   L.off_mstage = take(full ? C : 0);
   L.off_dhstage = take(full ? C * L.H * 4 : 0);
   L.off_rlstage = take(full ? C * 4 : 0);
+  L.off_list = take(full ? (size_t)L.N * 4 : 0);  // valid rows of a masked call, compacted
   L.off_dlog = take(full ? (size_t)L.G * C * L.Vp * 2 : 0);
   L.total = off;
   return L;
@@ -190,12 +191,12 @@ int debug_skip_commit() {
 // ---------------------------------------------------------------- profiling
 enum Kind {
   K_COUNT, K_PREP, K_FWD, K_MERGE, K_BWD, K_DH, K_DW, K_FINAL, K_ENT, K_ENT_MERGE, K_GATHER,
-  K_SCATTER, K_SELECT, K_NKINDS
+  K_SCATTER, K_SELECT, K_ZERO_DW, K_NKINDS
 };
 const char* const kKindName[K_NKINDS] = {
     "count_valid", "prep_teacher", "fwd_logits_lse", "merge_loss", "bwd_dlogits",
     "dH_gemm",     "dW_gemm",      "finalize",       "entropy_gemm", "merge_entropy",
-    "gather_rows", "scatter_rows", "select_rows"};
+    "gather_rows", "scatter_rows", "select_rows", "zero_dw"};
 struct ProfRec {
   int kind;
   cudaEvent_t a, b;
@@ -284,7 +285,7 @@ fckl_status run(const Request& q) {
   const fckl_problem* prob = q.prob;
   const bool bwd = q.mode == Mode::kFwdBwd;
   const bool ent = q.mode == Mode::kEntropy;
-  const bool list = q.rows != nullptr;
+  const bool user_list = q.rows != nullptr;
   if (!valid_problem(prob)) return FCKL_ERR_INVALID_ARG;
   if (!q.hidden || !q.W || !aligned(q.hidden, 16) || !aligned(q.W, 16)) return FCKL_ERR_INVALID_ARG;
   if (ent) {
@@ -297,7 +298,7 @@ fckl_status run(const Request& q) {
   }
   if (bwd && (!q.dH || !q.dW || !aligned(q.dH, 16) || !aligned(q.dW, 16)))
     return FCKL_ERR_INVALID_ARG;
-  if (list && (q.n_rows < 1 || q.n_rows > INT32_MAX || !aligned(q.rows, 4)))
+  if (user_list && (q.n_rows < 1 || q.n_rows > INT32_MAX || !aligned(q.rows, 4)))
     return FCKL_ERR_INVALID_ARG;
   if (!supported_problem(prob)) return FCKL_ERR_UNSUPPORTED;
   const Layout L = make_layout(prob, q.full_layout);
@@ -306,6 +307,16 @@ fckl_status run(const Request& q) {
   const DeviceInfo* dev = device_info();
   if (dev == nullptr || !dev->ok) return FCKL_ERR_UNSUPPORTED;
   if (get_encode_fn() == nullptr) return FCKL_ERR_CUDA;
+
+  // How the rows are fed to the chunk pipeline:
+  //   direct  : rows 0..N-1 in place (no mask, the entropy pass, or the
+  //             forward-only layout of the allocation-free entry point);
+  //   listed  : the caller's row list, gathered chunk by chunk;
+  //   compact : a masked call -- the valid rows are compacted on the device and
+  //             gathered, so masked rows cost no GEMM work; the row count of
+  //             each chunk is read on the device.
+  const bool compact = !ent && !user_list && q.row_mask != nullptr && q.full_layout;
+  const bool list = user_list || compact;
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(q.stream);
   uint8_t* ws = static_cast<uint8_t*>(q.workspace);
@@ -325,7 +336,9 @@ fckl_status run(const Request& q) {
   uint8_t* mstage = ws + L.off_mstage;
   float* dhstage = reinterpret_cast<float*>(ws + L.off_dhstage);
   float* rlstage = reinterpret_cast<float*>(ws + L.off_rlstage);
+  int32_t* clist = reinterpret_cast<int32_t*>(ws + L.off_list);
   __nv_bfloat16* dlog = reinterpret_cast<__nv_bfloat16*>(ws + L.off_dlog);
+  const int32_t* rowlist = user_list ? q.rows : clist;
 
   const int H = (int)L.H, V = (int)L.V, K = (int)L.K;
   const float invT = 1.0f / prob->T;
@@ -334,14 +347,27 @@ fckl_status run(const Request& q) {
 
   if (cudaMemsetAsync(ctl, 0, sizeof(DeviceCtl), st) != cudaSuccess) return FCKL_ERR_CUDA;
   if (!ent) {
-    ProfScope ps(K_COUNT, st, 0.0, list ? q.n_rows * 4.0 : (q.row_mask ? (double)L.N : 0.0));
-    const int nv_total = (int)prob->n_valid_total;
-    if (list)
-      k_count_list<<<1, 1024, 0, st>>>(q.rows, q.n_rows, L.N, nv_total, ctl);
+    ProfScope ps(K_COUNT, st, 0.0,
+                 user_list ? q.n_rows * 4.0 : (q.row_mask ? L.N * (compact ? 5.0 : 1.0) : 0.0));
+    if (user_list)
+      k_count_list<<<1, 1024, 0, st>>>(q.rows, q.n_rows, L.N, (int)prob->n_valid_total, ctl);
+    else if (compact)
+      k_compact_mask<<<1, 1024, 0, st>>>(q.row_mask, L.N, (int)prob->n_valid_total, clist, ctl);
     else
-      k_count_valid<<<1, 1024, 0, st>>>(q.row_mask, L.N, nv_total, ctl);
+      k_count_valid<<<1, 1024, 0, st>>>(q.row_mask, L.N, (int)prob->n_valid_total, ctl);
   }
-  if (list) {  // rows that are not listed get zero row loss and zero dH
+  // The profiler's flop and byte counts follow the rows a launch really
+  // processes; for a compacted call it reads their number back once (profiling
+  // only -- the normal path never waits on the device).
+  long long prof_rows = -1;
+  if (compact && g_prof.on) {
+    int32_t n = 0;
+    if (cudaMemcpyAsync(&n, &ctl->n_rows, sizeof(n), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+      return FCKL_ERR_CUDA;
+    prof_rows = n;
+  }
+  if (list) {  // rows that are not processed get zero row loss and zero dH
     if (cudaMemsetAsync(rl, 0, (size_t)L.N * 4, st) != cudaSuccess) return FCKL_ERR_CUDA;
     if (bwd && cudaMemsetAsync(q.dH, 0, (size_t)L.N * L.H * 4, st) != cudaSuccess)
       return FCKL_ERR_CUDA;
@@ -357,17 +383,28 @@ fckl_status run(const Request& q) {
   const long long KBh = cdiv(L.H, BK);
   const long long NTh = cdiv(L.H, BN);
   const long long KBv = cdiv(L.V, BK);
-  const long long R = list ? q.n_rows : L.N;  // rows (or list entries) to process
+  const long long R = user_list ? q.n_rows : L.N;  // rows (or list entries), upper bound
   const long long nchunks = cdiv(R, L.C);
   const long long G = std::min<long long>(nchunks, L.G);
-  auto grid_for = [&](long long units) { return (int)(2 * std::min<long long>(pairs, units)); };
+  auto grid_for = [&](long long units) {
+    return (int)(2 * std::max<long long>(1, std::min<long long>(pairs, units)));
+  };
+  // Rows of the chunk starting at row0 (at most cap): a host number, or read on
+  // the device for compacted calls.
+  auto rows_of = [&](long long row0, long long cap) {
+    return compact ? RowCount{-1, ctl, (int)row0, (int)cap} : RowCount{(int)cap, ctl, 0, 0};
+  };
   for (long long c = 0; c < nchunks; ++c) {
     const long long row0 = c * L.C;
-    const int rows = (int)std::min(L.C, R - row0);
-    const long long MT = cdiv(rows, PM);
-    const int row_blocks = (int)cdiv(rows, ROW_WARPS);
+    const int cap = (int)std::min(L.C, R - row0);  // rows of the chunk (upper bound if compact)
+    const RowCount rc = rows_of(row0, cap);
+    // rows this chunk processes, as far as the host knows (profiling figures)
+    const double nr = prof_rows < 0 ? (double)cap
+                                    : (double)std::max(0LL, std::min<long long>(cap, prof_rows - row0));
+    const long long MT = cdiv(cap, PM);
+    const int row_blocks = (int)cdiv(cap, ROW_WARPS);
     // Sources and destinations of this chunk: the caller's rows directly, or
-    // the staging buffers the listed rows are gathered into.
+    // the staging buffers the listed / compacted rows are gathered into.
     const void* h_c;
     const int32_t* ids_c;
     const float* lg_c;
@@ -377,14 +414,15 @@ fckl_status run(const Request& q) {
     if (list) {
       __nv_bfloat16* hdst = hstage + (size_t)(c % G) * L.C * L.H;
       {
-        ProfScope ps(K_GATHER, st, 0.0, (double)rows * (L.H * 4.0 + K * 16.0 + 5.0));
-        k_gather_rows<<<rows, 128, 0, st>>>(q.rows + row0, rows, L.N, H, K,
-                                            static_cast<const __nv_bfloat16*>(q.hidden),
-                                            q.topk_idx, q.topk_logit, hdst, idstage, lgstage,
-                                            mstage);
+        ProfScope ps(K_GATHER, st, 0.0, nr * (L.H * 4.0 + K * 16.0 + 5.0));
+        k_gather_rows<<<cap, 128, 0, st>>>(
+            rowlist + row0, rc, L.N, H, K, static_cast<const __nv_bfloat16*>(q.hidden),
+            q.topk_idx, q.topk_logit, hdst, idstage, lgstage, mstage,
+            bwd ? reinterpret_cast<uint4*>(dlog + (size_t)(c % G) * L.C * L.Vp) : nullptr,
+            L.Vp / 8);
       }
-      h_c = hdst; ids_c = idstage; lg_c = lgstage; mask_c = mstage; rl_c = rlstage;
-      dH_c = dhstage;
+      h_c = hdst; ids_c = idstage; lg_c = lgstage; rl_c = rlstage; dH_c = dhstage;
+      mask_c = compact ? nullptr : mstage;  // compacted rows are all valid
     } else {
       h_c = static_cast<const uint8_t*>(q.hidden) + (size_t)row0 * L.H * 2;
       ids_c = q.topk_idx ? q.topk_idx + row0 * K : nullptr;
@@ -397,88 +435,87 @@ fckl_status run(const Request& q) {
     __nv_bfloat16* dlog_c = dlog + (size_t)(c % G) * L.C * L.Vp;
 
     CUtensorMap mapH_k;
-    if (!make_map(&mapH_k, h_c, L.H, rows, L.H * 2, BK, CM)) return FCKL_ERR_CUDA;
+    if (!make_map(&mapH_k, h_c, L.H, cap, L.H * 2, BK, CM)) return FCKL_ERR_CUDA;
     // Forward units are vocab-major so that concurrent pairs share W tiles.
-    SchedArgs sa_v{MT * NT, SCHED_VOCAB_MAJOR, (int)MT, (int)NT, (int)KBh, 1, 0};
+    SchedArgs sa_v{SCHED_VOCAB_MAJOR, (int)NT, (int)KBh, 1, 0, rc};
     const int Gv = grid_for(MT * NT);
-    const double gemm_flops = 2.0 * rows * (double)L.V * (double)L.H;
+    const double gemm_flops = 2.0 * nr * (double)L.V * (double)L.H;
 
     if (ent) {  // student entropy: forward GEMM with the entropy epilogue, then merge
-      EpiEntropy::Params pe{rows, V, 1, (int)NT, scale2, nullptr, nullptr, nullptr, part, upart};
+      EpiEntropy::Params pe{V, 1, (int)NT, scale2, nullptr, nullptr, nullptr, part, upart};
       {
-        ProfScope ps(K_ENT, st, gemm_flops, 2.0 * (rows + (double)L.V) * L.H + rows * NT * 12.0);
+        ProfScope ps(K_ENT, st, gemm_flops, 2.0 * (nr + (double)L.V) * L.H + nr * NT * 12.0);
         gemm_pair_kernel<EpiEntropy, false, false>
             <<<Gv, GEMM_THREADS, pair_smem_bytes<EpiEntropy>(), st>>>(mapH_k, mapW_k, mapW_k, pe,
                                                                       sa_v, ca);
       }
       {
-        ProfScope ps(K_ENT_MERGE, st, 0.0, rows * NT * 12.0 + rows * 5.0);
-        k_merge_entropy<<<row_blocks, ROW_WARPS * 32, 0, st>>>(part, upart, (int)NT, rows, mask_c,
+        ProfScope ps(K_ENT_MERGE, st, 0.0, nr * NT * 12.0 + nr * 5.0);
+        k_merge_entropy<<<row_blocks, ROW_WARPS * 32, 0, st>>>(part, upart, (int)NT, rc, mask_c,
                                                                q.entropy + row0);
       }
       continue;
     }
 
     {
-      ProfScope ps(K_PREP, st, 0.0, (double)rows * K * 20.0 + rows * (NT + 1) * 2.0);
+      ProfScope ps(K_PREP, st, 0.0, nr * K * 20.0 + nr * (NT + 1) * 2.0);
       k_prep_teacher<<<row_blocks, ROW_WARPS * 32, 0, st>>>(
-          ids_c, lg_c, mask_c, rows, K, V, (int)NT, invT, prob->teacher == FCKL_TEACHER_PROBS,
+          ids_c, lg_c, mask_c, rc, K, V, (int)NT, invT, prob->teacher == FCKL_TEACHER_PROBS,
           sid, sp, zs, tstart, plogp, ctl);
     }
-    EpiLse::Params pf{rows, V, K, (int)NT, scale2, sid, tstart, zs, part, nullptr};
+    EpiLse::Params pf{V, K, (int)NT, scale2, sid, tstart, zs, part, nullptr};
     CtlArgs ca_f = ca;
     ca_f.debug_skip_commit = (c == 0) ? ca.debug_skip_commit : 0;
     {
-      ProfScope ps(K_FWD, st, gemm_flops, 2.0 * (rows + (double)L.V) * L.H + rows * NT * 8.0);
+      ProfScope ps(K_FWD, st, gemm_flops, 2.0 * (nr + (double)L.V) * L.H + nr * NT * 8.0);
       gemm_pair_kernel<EpiLse, false, false>
           <<<Gv, GEMM_THREADS, pair_smem_bytes<EpiLse>(), st>>>(mapH_k, mapW_k, mapW_k, pf, sa_v,
                                                                 ca_f);
     }
     {
-      ProfScope ps(K_MERGE, st, 0.0, (double)rows * K * 8.0 + rows * NT * 8.0 + rows * 13.0);
-      k_merge_loss<<<row_blocks, ROW_WARPS * 32, 0, st>>>(part, (int)NT, rows, K, invT, zs, sp,
+      ProfScope ps(K_MERGE, st, 0.0, nr * K * 8.0 + nr * NT * 8.0 + nr * 13.0);
+      k_merge_loss<<<row_blocks, ROW_WARPS * 32, 0, st>>>(part, (int)NT, rc, K, invT, zs, sp,
                                                            plogp, mask_c, lse2, rl_c);
     }
     if (!bwd) {
       if (list) {
-        ProfScope ps(K_SCATTER, st, 0.0, rows * 12.0);
-        k_scatter_rows<<<rows, 128, 0, st>>>(q.rows + row0, rows, L.N, H, rlstage, rl, nullptr,
-                                             nullptr);
+        ProfScope ps(K_SCATTER, st, 0.0, nr * 12.0);
+        k_scatter_rows<<<cap, 128, 0, st>>>(rowlist + row0, rc, L.N, H, rlstage, rl, nullptr,
+                                            nullptr);
       }
       continue;
     }
 
     // Backward 1: recompute the tiles and form bf16 dlogits = q - p~.
-    EpiDlogits::Params pb{rows, V, K, (int)NT, scale2, lse2, sid, tstart, sp, mask_c};
+    EpiDlogits::Params pb{V, K, (int)NT, scale2, lse2, sid, tstart, sp, mask_c};
     CUtensorMap mapD_st;
-    if (!make_map(&mapD_st, dlog_c, L.V, rows, L.Vp * 2, 64, 32)) return FCKL_ERR_CUDA;
+    if (!make_map(&mapD_st, dlog_c, L.V, cap, L.Vp * 2, 64, 32)) return FCKL_ERR_CUDA;
     {
-      ProfScope ps(K_BWD, st, gemm_flops, 2.0 * (rows + (double)L.V) * L.H + 2.0 * rows * L.V);
+      ProfScope ps(K_BWD, st, gemm_flops, 2.0 * (nr + (double)L.V) * L.H + 2.0 * nr * L.V);
       gemm_pair_kernel<EpiDlogits, false, false>
           <<<Gv, GEMM_THREADS, pair_smem_bytes<EpiDlogits>(), st>>>(mapH_k, mapW_k, mapD_st, pb,
                                                                     sa_v, ca);
     }
 
     // Backward 2: dH[rows] = alpha * dlogits W; A = dlogits (K-major), B = W (MN-major).
-    if (cudaMemsetAsync(dH_c, 0, (size_t)rows * L.H * 4, st) != cudaSuccess) return FCKL_ERR_CUDA;
+    if (cudaMemsetAsync(dH_c, 0, (size_t)cap * L.H * 4, st) != cudaSuccess) return FCKL_ERR_CUDA;
     CUtensorMap mapD_k, mapD_mn, mapH_mn, mapdH;
-    if (!make_map(&mapD_k, dlog_c, L.V, rows, L.Vp * 2, BK, CM)) return FCKL_ERR_CUDA;
-    if (!make_map(&mapdH, dH_c, L.H, rows, L.H * 4, 32, 32, true)) return FCKL_ERR_CUDA;
+    if (!make_map(&mapD_k, dlog_c, L.V, cap, L.Vp * 2, BK, CM)) return FCKL_ERR_CUDA;
+    if (!make_map(&mapdH, dH_c, L.H, cap, L.H * 4, 32, 32, true)) return FCKL_ERR_CUDA;
     const long long tiles_h = MT * NTh;
     const int S = choose_split(tiles_h, KBv, pairs);
-    SchedArgs sa_h{tiles_h * S, SCHED_SPLIT_K, (int)MT, (int)NTh, (int)KBv, S, (int)tiles_h};
-    EpiDH::Params ph{rows, H, invT, ctl};
+    SchedArgs sa_h{SCHED_SPLIT_K, (int)NTh, (int)KBv, S, 0, rc};
+    EpiDH::Params ph{H, invT, ctl};
     {
       ProfScope ps(K_DH, st, gemm_flops,
-                   2.0 * rows * (double)L.V + 2.0 * (double)L.V * L.H + 4.0 * rows * L.H);
+                   2.0 * nr * (double)L.V + 2.0 * (double)L.V * L.H + 4.0 * nr * L.H);
       gemm_pair_kernel<EpiDH, false, true>
           <<<grid_for(tiles_h * S), GEMM_THREADS, pair_smem_bytes<EpiDH>(), st>>>(
               mapD_k, mapW_mn, mapdH, ph, sa_h, ca);
     }
     if (list) {
-      ProfScope ps(K_SCATTER, st, 0.0, rows * (12.0 + 8.0 * L.H));
-      k_scatter_rows<<<rows, 128, 0, st>>>(q.rows + row0, rows, L.N, H, rlstage, rl, dhstage,
-                                           q.dH);
+      ProfScope ps(K_SCATTER, st, 0.0, nr * (12.0 + 8.0 * L.H));
+      k_scatter_rows<<<cap, 128, 0, st>>>(rowlist + row0, rc, L.N, H, rlstage, rl, dhstage, q.dH);
     }
 
     // Backward 3, once per group of G chunks (or at the last chunk):
@@ -487,17 +524,25 @@ fckl_status run(const Request& q) {
     if ((c + 1) % G != 0 && c + 1 != nchunks) continue;
     const long long g0 = c / G * G;  // first chunk of the group
     const long long grow0 = g0 * L.C;
-    const int grows = (int)(row0 + rows - grow0);
+    const int gcap = (int)(row0 + cap - grow0);
     const void* h_g = list ? static_cast<const void*>(hstage)
                            : static_cast<const uint8_t*>(q.hidden) + (size_t)grow0 * L.H * 2;
-    if (!make_map(&mapD_mn, dlog, L.V, grows, L.Vp * 2, 64, BK)) return FCKL_ERR_CUDA;
-    if (!make_map(&mapH_mn, h_g, L.H, grows, L.H * 2, 64, BK)) return FCKL_ERR_CUDA;
+    if (!make_map(&mapD_mn, dlog, L.V, gcap, L.Vp * 2, 64, BK)) return FCKL_ERR_CUDA;
+    if (!make_map(&mapH_mn, h_g, L.H, gcap, L.H * 2, 64, BK)) return FCKL_ERR_CUDA;
     const long long tiles_w = cdiv(L.V, PM) * NTh;
-    SchedArgs sa_w{tiles_w, SCHED_TILES, 0, (int)NTh, (int)cdiv(grows, BK), 1, (int)tiles_w};
+    SchedArgs sa_w{SCHED_TILES, (int)NTh, 0, 1, (int)cdiv(L.V, PM), rows_of(grow0, gcap)};
     EpiDW::Params pw{V, H, invT, g0 > 0 ? 1 : 0, ctl};
+    if (compact && g0 == 0) {  // with no valid row no dW launch below writes dW
+      ProfScope ps(K_ZERO_DW, st, 0.0, 0.0);
+      k_zero_if_no_valid<<<2 * pairs, 256, 0, st>>>(reinterpret_cast<float4*>(q.dW),
+                                                     L.V * L.H / 4, ctl);
+    }
     {
-      ProfScope ps(K_DW, st, 2.0 * grows * (double)L.V * (double)L.H,
-                   2.0 * grows * (double)L.V + 2.0 * grows * L.H +
+      const double gr = prof_rows < 0
+                            ? (double)gcap
+                            : (double)std::max(0LL, std::min<long long>(gcap, prof_rows - grow0));
+      ProfScope ps(K_DW, st, 2.0 * gr * (double)L.V * (double)L.H,
+                   2.0 * gr * (double)L.V + 2.0 * gr * L.H +
                        (g0 > 0 ? 8.0 : 4.0) * (double)L.V * L.H);
       gemm_pair_kernel<EpiDW, true, true>
           <<<grid_for(tiles_w), GEMM_THREADS, pair_smem_bytes<EpiDW>(), st>>>(

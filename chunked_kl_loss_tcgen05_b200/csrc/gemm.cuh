@@ -63,55 +63,81 @@ enum : uint32_t {
   SITE_DRAIN_MMA = 5, SITE_DRAIN_TMA = 6
 };
 
+// Rows a launch covers: a host value, or -- when the rows are the compacted
+// valid rows of a masked call, whose number only the device knows --
+// clamp(ctl->n_rows - row0, 0, cap), read when the kernel starts (the count is
+// written by an earlier kernel on the same stream).
+struct RowCount {
+  int fixed;  // >= 0: this many rows; < 0: read from ctl
+  const DeviceCtl* ctl;
+  int row0, cap;
+  __device__ __forceinline__ int get() const {
+    if (fixed >= 0) return fixed;
+    const int r = ctl->n_rows - row0;
+    return r < 0 ? 0 : (r > cap ? cap : r);
+  }
+};
+
 struct Work {
   int mt, nt;    // pair tile: rows [mt*256, +256), columns [nt*256, +256)
   int kb0, kb1;  // k-blocks [kb0, kb1) of 64
   int m0, n0;    // this CTA's first row (mt*256 + 128*rank) and the first column
+  int rows;      // rows of the launch (row-tiled kernels: rows >= rows are padding)
 };
 
 enum SchedKind : int {
   SCHED_VOCAB_MAJOR = 0,  // units (vocab tile nt, row tile mt), mt fastest; full K
   SCHED_SPLIT_K = 1,      // units (k segment, output tile), k segment slowest
-  SCHED_TILES = 2,        // units (mt, nt), nt fastest; full K
+  SCHED_TILES = 2,        // units (mt, nt), nt fastest; K = the launch's rows
 };
 
 struct SchedArgs {
-  long long total;  // number of units
   int kind;
-  int MT;           // row tiles (SCHED_VOCAB_MAJOR)
-  int NT;           // column tiles (SCHED_SPLIT_K, SCHED_TILES)
-  int KB;           // k-blocks of the full reduction
-  int S;            // split-K factor
-  int tiles;        // output tiles (SCHED_SPLIT_K)
+  int NT;      // vocab tiles (SCHED_VOCAB_MAJOR) / column tiles (SCHED_SPLIT_K, SCHED_TILES)
+  int KB;      // k-blocks of the reduction (SCHED_VOCAB_MAJOR, SCHED_SPLIT_K)
+  int S;       // split-K factor (SCHED_SPLIT_K)
+  int MT;      // row tiles of M (SCHED_TILES: M is the vocabulary)
+  RowCount rc; // the launch's rows: M of the first two kinds, K of SCHED_TILES
 };
 
 // Cluster c of G takes units c, c+G, c+2G, ...  In every order above, the
 // clusters running at the same moment touch a narrow band of the streamed
 // operand, so it is read from DRAM about once and reused from L2.
 struct PairSched {
-  long long u;
+  long long u, total;
   SchedArgs a;
-  int G;
+  int G, rows, MT, tiles, KB;
   __device__ void init(const SchedArgs& args, int cluster, int nclusters) {
     a = args; G = nclusters; u = cluster;
+    rows = a.rc.get();
+    const int row_tiles = (rows + PM - 1) / PM;
+    if (a.kind == SCHED_VOCAB_MAJOR) {
+      MT = row_tiles; KB = a.KB; tiles = MT * a.NT; total = (long long)tiles;
+    } else if (a.kind == SCHED_SPLIT_K) {
+      MT = row_tiles; KB = a.KB; tiles = MT * a.NT; total = (long long)tiles * a.S;
+    } else {
+      MT = a.MT; KB = (rows + BK - 1) / BK; tiles = MT * a.NT;
+      total = rows > 0 ? (long long)tiles : 0;
+    }
   }
   __device__ bool next(Work& w) {
-    if (u >= a.total) return false;
+    if (u >= total) return false;
     if (a.kind == SCHED_VOCAB_MAJOR) {
-      w.nt = (int)(u / a.MT);
-      w.mt = (int)(u - (long long)w.nt * a.MT);
-      w.kb0 = 0; w.kb1 = a.KB;
+      w.nt = (int)(u / MT);
+      w.mt = (int)(u - (long long)w.nt * MT);
+      w.kb0 = 0; w.kb1 = KB;
     } else if (a.kind == SCHED_SPLIT_K) {
-      const int ks = (int)(u / a.tiles);
-      const int tile = (int)(u - (long long)ks * a.tiles);
+      const int ks = (int)(u / tiles);
+      const int tile = (int)(u - (long long)ks * tiles);
       w.mt = tile / a.NT; w.nt = tile - w.mt * a.NT;
-      w.kb0 = (int)((long long)ks * a.KB / a.S);
-      w.kb1 = (int)((long long)(ks + 1) * a.KB / a.S);
+      w.kb0 = (int)((long long)ks * KB / a.S);
+      w.kb1 = (int)((long long)(ks + 1) * KB / a.S);
     } else {
       w.mt = (int)(u / a.NT);
       w.nt = (int)(u - (long long)w.mt * a.NT);
-      w.kb0 = 0; w.kb1 = a.KB;
+      w.kb0 = 0; w.kb1 = KB;
     }
+    w.rows = rows;
     u += G;
     return true;
   }
@@ -277,9 +303,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
-      // Every MMA issued by this thread is complete before TMEM is released.
-      umma_commit_pair(smem_u32(drain), 0x1);
-      drain_phase(smem_u32(drain), 0, wc, SITE_DRAIN_MMA);
+      // Every MMA issued by this thread is complete before TMEM is released
+      // (a pair with no unit -- a launch over zero device-counted rows -- issued none).
+      if ((long long)cluster < sch.total) {
+        umma_commit_pair(smem_u32(drain), 0x1);
+        drain_phase(smem_u32(drain), 0, wc, SITE_DRAIN_MMA);
+      }
     }
     __syncwarp();
   } else {

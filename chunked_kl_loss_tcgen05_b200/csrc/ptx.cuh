@@ -19,7 +19,8 @@ struct DeviceCtl {
   uint32_t err;       // OR of kErr* bits
   int32_t n_valid;    // number of rows with row_mask != 0
   uint32_t timeout_site;  // which wait gave up first (diagnostics)
-  uint32_t pad[61];
+  int32_t n_rows;     // rows a masked call compacted (its local valid rows)
+  uint32_t pad[60];
 };
 static_assert(sizeof(DeviceCtl) == 256, "control block is 256 bytes");
 

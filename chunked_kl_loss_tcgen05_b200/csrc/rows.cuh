@@ -72,16 +72,47 @@ __global__ void __launch_bounds__(1024) k_count_list(const int32_t* __restrict__
   }
 }
 
+// Row indices of the valid rows (row_mask != 0), ascending, into list[0, n),
+// n into ctl->n_rows and N_v (n, or the caller's global total when > 0) into
+// ctl->n_valid.  One block: each thread scans a contiguous range; a block-wide
+// prefix sum gives every thread its output position.
+__global__ void __launch_bounds__(1024) k_compact_mask(const uint8_t* __restrict__ mask,
+                                                       long long N, int total,
+                                                       int32_t* __restrict__ list, DeviceCtl* ctl);
+
+// dW = 0 when the call compacted no row (then no dW launch writes it);
+// otherwise nothing.
+__global__ void k_zero_if_no_valid(float4* __restrict__ out, long long n4, const DeviceCtl* ctl) {
+  if (ctl->n_rows > 0) return;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4;
+       i += (long long)gridDim.x * blockDim.x)
+    out[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
 // Gather the listed rows of one chunk (block i copies list entry i): hidden
 // row -> hst[i] (bf16, 16-byte vectors), teacher ids/logits -> idst/lgst[i],
 // mst[i] = 1.  Entries outside [0, N) give a zero row with mst[i] = 0.
+// When the row count n is read on the device (fewer rows than the launch's
+// blocks), blocks n .. n+63 zero their staged hidden row and, if dlz is given,
+// their dlogits row (dl_u4 16-byte words each): the dW GEMM reads whole blocks
+// of 64 rows, and the rows past n that its last block covers must be zero.
 __global__ void __launch_bounds__(128)
-    k_gather_rows(const int32_t* __restrict__ list, int rows_c, long long N, int H, int K,
+    k_gather_rows(const int32_t* __restrict__ list, RowCount rc, long long N, int H, int K,
                   const __nv_bfloat16* __restrict__ hidden, const int32_t* __restrict__ ids,
                   const float* __restrict__ lg, __nv_bfloat16* __restrict__ hst,
-                  int32_t* __restrict__ idst, float* __restrict__ lgst, uint8_t* __restrict__ mst) {
+                  int32_t* __restrict__ idst, float* __restrict__ lgst, uint8_t* __restrict__ mst,
+                  uint4* __restrict__ dlz, long long dl_u4) {
   const int i = blockIdx.x;
-  if (i >= rows_c) return;
+  const int n = rc.get();
+  if (i >= n) {
+    if (i >= n + 64) return;
+    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+    uint4* hrow = reinterpret_cast<uint4*>(hst + (size_t)i * H);
+    for (int j = threadIdx.x; j < H / 8; j += blockDim.x) hrow[j] = zero;
+    if (dlz != nullptr)
+      for (long long j = threadIdx.x; j < dl_u4; j += blockDim.x) dlz[(size_t)i * dl_u4 + j] = zero;
+    return;
+  }
   const int r = list[i];
   const bool ok = r >= 0 && r < N;
   const uint4* src = reinterpret_cast<const uint4*>(hidden + (size_t)(ok ? r : 0) * H);
@@ -98,11 +129,11 @@ __global__ void __launch_bounds__(128)
 // Scatter one chunk's per-entry results back to the listed rows: row loss and
 // (when dH is given) the fp32 dH row.
 __global__ void __launch_bounds__(128)
-    k_scatter_rows(const int32_t* __restrict__ list, int rows_c, long long N, int H,
+    k_scatter_rows(const int32_t* __restrict__ list, RowCount rc, long long N, int H,
                    const float* __restrict__ rl_stage, float* __restrict__ rl,
                    const float* __restrict__ dh_stage, float* __restrict__ dH) {
   const int i = blockIdx.x;
-  if (i >= rows_c) return;
+  if (i >= rc.get()) return;
   const int r = list[i];
   if (r < 0 || r >= N) return;
   if (threadIdx.x == 0) rl[r] = rl_stage[i];
@@ -143,6 +174,24 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* sh, int* total) 
   *total = sh[(blockDim.x >> 5) - 1];
   __syncthreads();
   return before;
+}
+
+__global__ void __launch_bounds__(1024) k_compact_mask(const uint8_t* __restrict__ mask,
+                                                       long long N, int total,
+                                                       int32_t* __restrict__ list, DeviceCtl* ctl) {
+  __shared__ int sh[32];
+  const long long per = (N + blockDim.x - 1) / blockDim.x;
+  const long long i0 = threadIdx.x * per, i1 = (i0 + per < N) ? i0 + per : N;
+  int cnt = 0;
+  for (long long i = i0; i < i1; ++i) cnt += mask[i] != 0;
+  int count;
+  int pos = block_exclusive_scan(cnt, sh, &count);
+  for (long long i = i0; i < i1; ++i)
+    if (mask[i] != 0) list[pos++] = (int32_t)i;
+  if (threadIdx.x == 0) {
+    ctl->n_rows = count;
+    ctl->n_valid = total > 0 ? total : count;
+  }
 }
 
 // Top-n rows by score among valid rows (row_mask != 0, or all), one block:
@@ -233,7 +282,7 @@ __global__ void __launch_bounds__(1024)
 // by INT_MAX, which no vocab column matches.
 __global__ void __launch_bounds__(ROW_WARPS * 32)
     k_prep_teacher(const int32_t* __restrict__ ids, const float* __restrict__ lg,
-                   const uint8_t* __restrict__ mask, int rows_c, int K, int V, int NT,
+                   const uint8_t* __restrict__ mask, RowCount rc, int K, int V, int NT,
                    float invT, bool probs, int* __restrict__ sid, float* __restrict__ sp,
                    float* __restrict__ zs, uint16_t* __restrict__ tstart,
                    float* __restrict__ plogp, DeviceCtl* ctl) {
@@ -242,7 +291,7 @@ __global__ void __launch_bounds__(ROW_WARPS * 32)
   __shared__ float s_sp[ROW_WARPS][K_MAX];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * ROW_WARPS + warp;
-  if (row >= rows_c) return;  // warp-uniform
+  if (row >= rc.get()) return;  // warp-uniform
   const bool keep = mask == nullptr || mask[row] != 0;
   float t[K_MAX / 32];
   int id[K_MAX / 32];
@@ -342,13 +391,13 @@ __global__ void __launch_bounds__(ROW_WARPS * 32)
 // log-sum-exp (log2 domain, kept for the backward epilogue) and form the row
 // loss  l_r = sum_k p_k log p_k - sum_k p_k (z_k / T - LSE_r),  0 for masked rows.
 __global__ void __launch_bounds__(ROW_WARPS * 32)
-    k_merge_loss(const float2* __restrict__ partials, int NT, int rows_c, int K, float invT,
+    k_merge_loss(const float2* __restrict__ partials, int NT, RowCount rc, int K, float invT,
                  const float* __restrict__ zs, const float* __restrict__ sp,
                  const float* __restrict__ plogp, const uint8_t* __restrict__ mask,
                  float* __restrict__ lse2_out, float* __restrict__ row_loss) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * ROW_WARPS + warp;
-  if (row >= rows_c) return;
+  if (row >= rc.get()) return;
   const float2* pr = partials + (size_t)row * NT;
   float M = -INFINITY;
   for (int t = lane; t < NT; t += 32) M = fmaxf(M, pr[t].x);
@@ -380,10 +429,10 @@ __global__ void __launch_bounds__(ROW_WARPS * 32)
 // Masked rows get 0.
 __global__ void __launch_bounds__(ROW_WARPS * 32)
     k_merge_entropy(const float2* __restrict__ partials, const float* __restrict__ upart, int NT,
-                    int rows_c, const uint8_t* __restrict__ mask, float* __restrict__ entropy) {
+                    RowCount rc, const uint8_t* __restrict__ mask, float* __restrict__ entropy) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * ROW_WARPS + warp;
-  if (row >= rows_c) return;
+  if (row >= rc.get()) return;
   const float2* pr = partials + (size_t)row * NT;
   const float* pu = upart + (size_t)row * NT;
   float M = -INFINITY;

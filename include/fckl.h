@@ -117,8 +117,9 @@ typedef enum { FCKL_TEACHER_LOGITS = 0, FCKL_TEACHER_PROBS = 1 } fckl_teacher_fo
 
 /* Bytes of device workspace fckl_fwd / fckl_fwd_bwd / fckl_fwd_bwd_rows /
  * fckl_student_entropy need for `prob` (0 when the problem is invalid): the
- * per-chunk teacher, log-sum-exp and dlogits buffers, N floats of row loss
- * and the staging buffers row-list calls gather into.  Pure host arithmetic;
+ * per-chunk teacher, log-sum-exp and dlogits buffers, N floats of row loss,
+ * N int32 of compacted row list and the staging buffers that row-list and
+ * masked calls gather into.  Pure host arithmetic;
  * needs no GPU. */
 size_t fckl_workspace_bytes(const fckl_problem* prob);
 
@@ -130,7 +131,9 @@ int64_t fckl_resolved_chunk(const fckl_problem* prob);
  * over the K cached logits, the fused projection z = h W^T on the tensor cores
  * with a full-vocabulary online log-sum-exp and a gather of z at the cached
  * ids (the [chunk, V] logit tile is never written), then the per-row KL.
- * Cost: 2*H*V flops per row. */
+ * With a row_mask, the valid rows are first compacted on the device and
+ * gathered chunk by chunk, so masked rows cost no GEMM work (row_loss is 0
+ * there).  Cost: 2*H*V flops per valid row. */
 fckl_status fckl_fwd(const fckl_problem* prob, const void* hidden, const void* W,
                      const int32_t* topk_idx, const float* topk_logit,
                      const uint8_t* row_mask, float* loss, float* row_loss,
@@ -140,7 +143,8 @@ fckl_status fckl_fwd(const fckl_problem* prob, const void* hidden, const void* W
  * Per chunk, after the forward steps above: recompute the logit tile, form
  * bf16 dlogits = q - p~ (masked rows 0) in the GEMM epilogue, then
  * dH_chunk = (1/(T N_v)) dlogits W and dW += (1/(T N_v)) dlogits^T h_chunk on
- * the tensor cores with fp32 accumulation.  Cost: 8*H*V flops per row. */
+ * the tensor cores with fp32 accumulation; masked rows are skipped as in
+ * fckl_fwd (their dH rows are 0).  Cost: 8*H*V flops per valid row. */
 fckl_status fckl_fwd_bwd(const fckl_problem* prob, const void* hidden, const void* W,
                          const int32_t* topk_idx, const float* topk_logit,
                          const uint8_t* row_mask, float* loss, float* row_loss,
@@ -241,9 +245,13 @@ const char* fckl_status_string(fckl_status status);
  * per-kernel summaries (one per kind, in first-launch order); it returns how
  * many kinds were seen, or -1 on a CUDA error.  Recording is process-wide and
  * not thread-safe.
+ * A masked call's flop and byte figures count the rows it processes (its
+ * valid rows); to know their number it reads one integer back from the device
+ * once per call while recording is on.
  * Kinds: 0 count_valid, 1 prep_teacher, 2 fwd_logits_lse, 3 merge_loss,
  *        4 bwd_dlogits, 5 dH_gemm, 6 dW_gemm, 7 finalize, 8 entropy_gemm,
- *        9 merge_entropy, 10 gather_rows, 11 scatter_rows, 12 select_rows. */
+ *        9 merge_entropy, 10 gather_rows, 11 scatter_rows, 12 select_rows,
+ *        13 zero_dw. */
 typedef struct {
   char name[32];     /* kernel kind, e.g. "fwd_logits_lse" */
   int64_t launches;  /* launches recorded */

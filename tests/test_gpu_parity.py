@@ -127,6 +127,38 @@ def test_masked_rows_do_not_matter():
     assert g2["dH"][torch.from_numpy(m).cuda()].abs().max().item() == 0.0
 
 
+def _with_valid_count(inp, n_valid, seed):
+    rng = np.random.default_rng(seed)
+    m = np.zeros(inp.cfg.N, np.uint8)
+    m[rng.choice(inp.cfg.N, size=n_valid, replace=False)] = 1
+    inp.row_mask[:] = m
+    return inp
+
+
+@pytest.mark.parametrize("n_valid", [1, 63, 100, 150, 190, 299])
+@pytest.mark.parametrize("fill", [0x00, 0xFF])
+def test_compacted_rows_against_oracle(n_valid, fill):
+    """Masked calls compact their valid rows on the device.  Chunk 100 (not a
+    multiple of 64) with three chunks per dW group puts the partial 64-row block
+    of the dW reduction across chunk slots for some counts; a workspace filled
+    with 0xFF bytes (NaN in bf16 and fp32) shows that no stale value leaks in."""
+    inp = _with_valid_count(synth.make_custom(300, 64, 700, 9, T=1.2, sigma=2.0, seed=21,
+                                              chunk=100), n_valid, n_valid)
+    o = oracle.oracle_from_inputs(inp)
+    d = arrays_to_device(inp.hidden, inp.W, inp.topk_idx, inp.topk_logit, inp.row_mask)
+    prob = FcklProblem(300, 64, 700, 9, 1.2, 100)
+    ws = alloc_workspace(prob, d[0].device)
+    ws.fill_(fill)
+    loss, rl, dH, dW = fused_kl_fwd_bwd(*d, T=1.2, chunk=100, workspace=ws, want_row_loss=True)
+    torch.cuda.synchronize()
+    check_full(inp, dict(loss=loss.item(), row_loss=rl.cpu().numpy(), dH=dH, dW=dW), o)
+    ws.fill_(fill)
+    lf, rlf = fused_kl_fwd(*d, T=1.2, chunk=100, workspace=ws, want_row_loss=True)
+    torch.cuda.synchronize()
+    assert lf.item() == pytest.approx(loss.item(), rel=1e-6)
+    np.testing.assert_allclose(rlf.cpu().numpy(), rl.cpu().numpy(), rtol=1e-6, atol=1e-7)
+
+
 def test_llama_8k_config_full():
     inp = synth.make_inputs(1)
     g = run_gpu(inp)
