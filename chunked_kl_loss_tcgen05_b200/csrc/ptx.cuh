@@ -77,9 +77,8 @@ __device__ __forceinline__ void raise_timeout(const WaitCtx& w, uint32_t site) {
 // Waits for completion of the phase with parity `parity`.  Returns false (and
 // raises the abort flag) when the budget runs out, or when another role of the
 // CTA has already aborted.  Never spins without limit.
-__device__ __noinline__ bool wait_phase(uint32_t bar, uint32_t parity, const WaitCtx& w,
-                                        uint32_t site) {
-  if (mbar_try_wait(bar, parity)) return true;
+__device__ __noinline__ bool wait_phase_slow(uint32_t bar, uint32_t parity, const WaitCtx& w,
+                                             uint32_t site) {
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -91,6 +90,14 @@ __device__ __noinline__ bool wait_phase(uint32_t bar, uint32_t parity, const Wai
       }
     }
   }
+}
+
+// The common case -- the phase has already completed -- stays inline; the
+// bounded loop is a call.
+__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, const WaitCtx& w,
+                                           uint32_t site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return wait_phase_slow(bar, parity, w, site);
 }
 
 // Cleanup wait: ignores the abort flag (it is used to let in-flight copies and
