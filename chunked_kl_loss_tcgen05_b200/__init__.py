@@ -21,6 +21,7 @@ __all__ = [
     "fckl_workspace_bytes", "fckl_resolved_chunk", "fckl_fwd", "fckl_fwd_bwd", "fckl_check",
     "fckl_status_string", "FcklKernelStat", "fckl_profile_begin", "fckl_profile_end",
     "fckl_fwd_noalloc", "fckl_student_entropy", "fckl_select_top_rows", "fckl_fwd_bwd_rows",
+    "fckl_host_workspace_bytes", "fckl_fwd_bwd_host",
 ]
 
 FCKL_OK = 0
@@ -39,7 +40,7 @@ _LIB = None
 exported_symbols = ("fckl_workspace_bytes", "fckl_resolved_chunk", "fckl_fwd", "fckl_fwd_bwd",
                     "fckl_check", "fckl_status_string", "fckl_profile_begin", "fckl_profile_end",
                     "fckl_fwd_noalloc", "fckl_student_entropy", "fckl_select_top_rows",
-                    "fckl_fwd_bwd_rows")
+                    "fckl_fwd_bwd_rows", "fckl_host_workspace_bytes", "fckl_fwd_bwd_host")
 
 
 FCKL_TEACHER_LOGITS = 0
@@ -94,6 +95,10 @@ def load() -> ctypes.CDLL:
     lib.fckl_fwd.restype = ctypes.c_int
     lib.fckl_fwd_bwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.fckl_fwd_bwd.restype = ctypes.c_int
+    lib.fckl_host_workspace_bytes.argtypes = [P]
+    lib.fckl_host_workspace_bytes.restype = sz
+    lib.fckl_fwd_bwd_host.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.fckl_fwd_bwd_host.restype = ctypes.c_int
     lib.fckl_check.argtypes = [vp, vp]
     lib.fckl_check.restype = ctypes.c_int
     lib.fckl_status_string.argtypes = [ctypes.c_int]
@@ -123,6 +128,10 @@ def fckl_workspace_bytes(prob: FcklProblem) -> int:
     return int(load().fckl_workspace_bytes(ctypes.byref(prob)))
 
 
+def fckl_host_workspace_bytes(prob: FcklProblem) -> int:
+    return int(load().fckl_host_workspace_bytes(ctypes.byref(prob)))
+
+
 def fckl_resolved_chunk(prob: FcklProblem) -> int:
     return int(load().fckl_resolved_chunk(ctypes.byref(prob)))
 
@@ -143,6 +152,17 @@ def fckl_fwd_bwd(prob, hidden, W, topk_idx, topk_logit, row_mask, loss, row_loss
                                    _ptr(topk_logit), _ptr(row_mask), _ptr(loss),
                                    _ptr(row_loss), _ptr(dH), _ptr(dW), _ptr(workspace),
                                    ctypes.c_size_t(int(workspace_bytes)), _ptr(stream)))
+
+
+def fckl_fwd_bwd_host(prob, hidden_host, W, topk_idx_host, topk_logit_host, row_mask_host,
+                      loss_host, dH, dW, workspace, workspace_bytes, stream) -> int:
+    """Inputs and the loss are HOST addresses (ints; row_mask may be None); W, dH,
+    dW and the workspace are device addresses.  Returns the status."""
+    return int(load().fckl_fwd_bwd_host(ctypes.byref(prob), _ptr(hidden_host), _ptr(W),
+                                        _ptr(topk_idx_host), _ptr(topk_logit_host),
+                                        _ptr(row_mask_host), _ptr(loss_host), _ptr(dH), _ptr(dW),
+                                        _ptr(workspace), ctypes.c_size_t(int(workspace_bytes)),
+                                        _ptr(stream)))
 
 
 def fckl_fwd_noalloc(prob, hidden, W, topk_idx, topk_logit, row_mask, loss, row_loss,

@@ -279,6 +279,9 @@ struct Request {
   size_t ws_bytes = 0;
   void* stream = nullptr;
   bool full_layout = true;
+  // Host-input calls: ready[0] marks the row mask copied to the device,
+  // ready[1 + c] the rows chunk c reads; the chunk waits for it on the stream.
+  const cudaEvent_t* ready = nullptr;
 };
 
 fckl_status run(const Request& q) {
@@ -346,6 +349,7 @@ fckl_status run(const Request& q) {
   CtlArgs ca{ctl, wait_timeout_ns(), debug_skip_commit()};
 
   if (cudaMemsetAsync(ctl, 0, sizeof(DeviceCtl), st) != cudaSuccess) return FCKL_ERR_CUDA;
+  if (q.ready && cudaStreamWaitEvent(st, q.ready[0], 0) != cudaSuccess) return FCKL_ERR_CUDA;
   if (!ent) {
     ProfScope ps(K_COUNT, st, 0.0,
                  user_list ? q.n_rows * 4.0 : (q.row_mask ? L.N * (compact ? 5.0 : 1.0) : 0.0));
@@ -395,6 +399,7 @@ fckl_status run(const Request& q) {
     return compact ? RowCount{-1, ctl, (int)row0, (int)cap} : RowCount{(int)cap, ctl, 0, 0};
   };
   for (long long c = 0; c < nchunks; ++c) {
+    if (q.ready && cudaStreamWaitEvent(st, q.ready[1 + c], 0) != cudaSuccess) return FCKL_ERR_CUDA;
     const long long row0 = c * L.C;
     const int cap = (int)std::min(L.C, R - row0);  // rows of the chunk (upper bound if compact)
     const RowCount rc = rows_of(row0, cap);
@@ -599,6 +604,52 @@ __global__ void k_export_status(const DeviceCtl* ctl, int32_t* status_out) {
 
 }  // namespace
 
+// ---------------------------------------------------------------- host inputs
+// Per device: a copy stream and a pool of events for the host-input entry
+// point (created on first use, kept until the process exits).
+struct HostIO {
+  std::mutex mu;
+  cudaStream_t cs = nullptr;
+  std::vector<cudaEvent_t> ev;
+};
+HostIO g_hio[kMaxDevices];
+
+// Device copies of the host inputs, after the regular workspace.
+struct HostLayout {
+  size_t off_hidden, off_ids, off_lg, off_mask, off_loss, total;
+};
+HostLayout make_host_layout(const fckl_problem* p) {
+  HostLayout h{};
+  size_t off = make_layout(p).total;
+  auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, kAlign); return o; };
+  h.off_hidden = take((size_t)p->N * p->H * 2);
+  h.off_ids = take((size_t)p->N * p->K * 4);
+  h.off_lg = take((size_t)p->N * p->K * 4);
+  h.off_mask = take((size_t)p->N);
+  h.off_loss = take(4);
+  h.total = off;
+  return h;
+}
+
+// Host rows [0, end[c]) hold every row chunk c reads: with a mask, chunk c
+// takes the valid rows numbered [c*C, (c+1)*C) (in row order), so end[c] is one
+// past the last of them; the piece that reaches the last valid row runs to N.
+std::vector<long long> piece_ends(const uint8_t* mask, long long N, long long C) {
+  const long long nchunks = cdiv(N, C);
+  std::vector<long long> end(nchunks, N);
+  if (mask == nullptr) {
+    for (long long c = 0; c < nchunks; ++c) end[c] = std::min(N, (c + 1) * C);
+    return end;
+  }
+  long long seen = 0, c = 0;
+  for (long long i = 0; i < N && c < nchunks; ++i) {
+    if (mask[i] == 0) continue;
+    if (++seen == (c + 1) * C) end[c++] = i + 1;
+  }
+  if (c < nchunks) end[c] = N;  // the chunk holding the last valid row (or none)
+  return end;
+}
+
 extern "C" {
 
 fckl_status fckl_fwd_noalloc(const fckl_problem* prob, const void* hidden, const void* W,
@@ -665,6 +716,89 @@ fckl_status fckl_fwd_bwd(const fckl_problem* prob, const void* hidden, const voi
   q.row_mask = row_mask; q.loss = loss; q.row_loss = row_loss; q.dH = dH; q.dW = dW;
   q.workspace = workspace; q.ws_bytes = workspace_bytes; q.stream = stream;
   return run(q);
+}
+
+size_t fckl_host_workspace_bytes(const fckl_problem* prob) {
+  if (!valid_problem(prob) || !supported_problem(prob)) return 0;
+  return make_host_layout(prob).total;
+}
+
+fckl_status fckl_fwd_bwd_host(const fckl_problem* prob, const void* hidden_host, const void* W,
+                              const int32_t* topk_idx_host, const float* topk_logit_host,
+                              const uint8_t* row_mask_host, float* loss_host, float* dH, float* dW,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+  if (!valid_problem(prob)) return FCKL_ERR_INVALID_ARG;
+  if (!hidden_host || !topk_idx_host || !topk_logit_host || !loss_host)
+    return FCKL_ERR_INVALID_ARG;
+  if (!supported_problem(prob)) return FCKL_ERR_UNSUPPORTED;
+  const HostLayout HL = make_host_layout(prob);
+  if (workspace == nullptr || !aligned(workspace, kAlign) || workspace_bytes < HL.total)
+    return FCKL_ERR_WORKSPACE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FCKL_ERR_CUDA;
+  const long long N = prob->N, H = prob->H, K = prob->K;
+  const long long C = resolve_chunk(prob);
+  const long long nchunks = cdiv(N, C);
+  const std::vector<long long> end = piece_ends(row_mask_host, N, C);
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* hid = ws + HL.off_hidden;
+  int32_t* ids = reinterpret_cast<int32_t*>(ws + HL.off_ids);
+  float* lg = reinterpret_cast<float*>(ws + HL.off_lg);
+  uint8_t* mask = row_mask_host ? ws + HL.off_mask : nullptr;
+  float* loss_dev = reinterpret_cast<float*>(ws + HL.off_loss);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+  HostIO& io = g_hio[dev];
+  std::lock_guard<std::mutex> lk(io.mu);
+  if (io.cs == nullptr && cudaStreamCreateWithFlags(&io.cs, cudaStreamNonBlocking) != cudaSuccess) {
+    io.cs = nullptr;
+    return FCKL_ERR_CUDA;
+  }
+  while ((long long)io.ev.size() < nchunks + 2) {
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return FCKL_ERR_CUDA;
+    io.ev.push_back(e);
+  }
+  // The copies start after the work already on the caller's stream (which may
+  // still read the device copies of a previous call).
+  auto ok = [](cudaError_t e) { return e == cudaSuccess; };
+  if (!ok(cudaEventRecord(io.ev[0], st)) || !ok(cudaStreamWaitEvent(io.cs, io.ev[0], 0)))
+    return FCKL_ERR_CUDA;
+  if (mask && !ok(cudaMemcpyAsync(mask, row_mask_host, (size_t)N, cudaMemcpyHostToDevice, io.cs)))
+    return FCKL_ERR_CUDA;
+  if (!ok(cudaEventRecord(io.ev[1], io.cs))) return FCKL_ERR_CUDA;
+  long long r0 = 0;
+  for (long long c = 0; c < nchunks; ++c) {
+    const long long r1 = end[c];
+    if (r1 > r0) {
+      const size_t n = (size_t)(r1 - r0);
+      if (!ok(cudaMemcpyAsync(hid + (size_t)r0 * H * 2,
+                              static_cast<const uint8_t*>(hidden_host) + (size_t)r0 * H * 2,
+                              n * H * 2, cudaMemcpyHostToDevice, io.cs)) ||
+          !ok(cudaMemcpyAsync(ids + (size_t)r0 * K, topk_idx_host + (size_t)r0 * K, n * K * 4,
+                              cudaMemcpyHostToDevice, io.cs)) ||
+          !ok(cudaMemcpyAsync(lg + (size_t)r0 * K, topk_logit_host + (size_t)r0 * K, n * K * 4,
+                              cudaMemcpyHostToDevice, io.cs)))
+        return FCKL_ERR_CUDA;
+      r0 = r1;
+    }
+    if (!ok(cudaEventRecord(io.ev[2 + c], io.cs))) return FCKL_ERR_CUDA;
+  }
+  Request q;
+  q.mode = Mode::kFwdBwd;
+  q.prob = prob; q.hidden = hid; q.W = W; q.topk_idx = ids; q.topk_logit = lg;
+  q.row_mask = mask; q.loss = loss_dev; q.dH = dH; q.dW = dW;
+  q.workspace = workspace; q.ws_bytes = workspace_bytes; q.stream = stream;
+  q.ready = io.ev.data() + 1;
+  const fckl_status s = run(q);
+  if (s != FCKL_OK) {
+    cudaStreamWaitEvent(st, io.ev[1 + nchunks], 0);  // leave no copy running past the call
+    return s;
+  }
+  if (!ok(cudaMemcpyAsync(loss_host, loss_dev, 4, cudaMemcpyDeviceToHost, st)))
+    return FCKL_ERR_CUDA;
+  return FCKL_OK;
 }
 
 fckl_status fckl_fwd_bwd_rows(const fckl_problem* prob, const void* hidden, const void* W,

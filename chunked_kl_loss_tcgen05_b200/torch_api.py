@@ -11,11 +11,12 @@ from __future__ import annotations
 import torch
 
 from . import (FcklError, FcklProblem, FCKL_OK, fckl_check, fckl_fwd, fckl_fwd_bwd,
-               fckl_workspace_bytes)
+               fckl_fwd_bwd_host, fckl_host_workspace_bytes, fckl_workspace_bytes)
 
 __all__ = ["make_problem", "alloc_workspace", "fused_kl_fwd", "fused_kl_fwd_bwd", "student_entropy",
            "select_top_rows", "fused_kl_rows", "arrays_to_device",
-           "fused_kl_from_host", "FusedChunkedKL", "fused_chunked_kl_loss"]
+           "fused_kl_from_host", "alloc_host_workspace", "fused_kl_fwd_bwd_host",
+           "FusedChunkedKL", "fused_chunked_kl_loss"]
 
 
 def _bits(t: torch.Tensor) -> torch.Tensor:
@@ -114,6 +115,59 @@ def fused_kl_fwd(hidden, W, topk_idx, topk_logit, row_mask=None, T=1.0, chunk=0,
         if st != FCKL_OK:
             raise FcklError(st, "fckl_check")
     return loss, row_loss
+
+
+def alloc_host_workspace(prob: FcklProblem, device) -> torch.Tensor:
+    nbytes = fckl_host_workspace_bytes(prob)
+    if nbytes == 0:
+        raise FcklError(1, "fckl_host_workspace_bytes")
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def fused_kl_fwd_bwd_host(hidden, W, topk_idx, topk_logit, row_mask=None, T=1.0, chunk=0,
+                          workspace=None, out=None, loss_host=None, check=True):
+    """Forward + backward from HOST inputs (contiguous CPU tensors; pinned for
+    overlapped copies): hidden bf16 [N,H], topk_idx int32 [N,K], topk_logit
+    float32 [N,K], row_mask uint8 [N] or None.  W is a CUDA bf16 tensor.  The
+    library streams the inputs to the device chunk by chunk, overlapped with
+    the kernels.  Returns (loss as a Python float, dH, dW); the loss read
+    synchronises the stream."""
+    hidden, W = _bits(hidden), _bits(W)
+    for name, t in (("hidden", hidden), ("topk_idx", topk_idx), ("topk_logit", topk_logit)):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CPU tensor")
+    if row_mask is not None and (row_mask.is_cuda or row_mask.dtype != torch.uint8
+                                 or not row_mask.is_contiguous()):
+        raise TypeError("row_mask must be a contiguous uint8 CPU tensor")
+    if not W.is_cuda or not W.is_contiguous():
+        raise ValueError("W must be a contiguous CUDA tensor")
+    if topk_idx.dtype != torch.int32 or topk_logit.dtype != torch.float32:
+        raise TypeError("topk_idx must be int32 and topk_logit float32")
+    prob = make_problem(hidden, W, topk_idx, T, chunk)
+    dev = W.device
+    if workspace is None:
+        workspace = alloc_host_workspace(prob, dev)
+    if out is None:
+        out = (torch.empty(prob.N, prob.H, dtype=torch.float32, device=dev),
+               torch.empty(prob.V, prob.H, dtype=torch.float32, device=dev))
+    dH, dW = out
+    if loss_host is None:
+        loss_host = torch.empty(1, dtype=torch.float32, pin_memory=True)
+    stream = torch.cuda.current_stream(dev)
+    st = fckl_fwd_bwd_host(prob, hidden.data_ptr(), W.data_ptr(), topk_idx.data_ptr(),
+                           topk_logit.data_ptr(),
+                           None if row_mask is None else row_mask.data_ptr(),
+                           loss_host.data_ptr(), dH.data_ptr(), dW.data_ptr(),
+                           workspace.data_ptr(), workspace.numel(), stream.cuda_stream)
+    if st != FCKL_OK:
+        raise FcklError(st, "fckl_fwd_bwd_host")
+    if check:
+        st = fckl_check(workspace.data_ptr(), stream.cuda_stream)
+        if st != FCKL_OK:
+            raise FcklError(st, "fckl_check")
+    else:
+        stream.synchronize()
+    return float(loss_host[0]), dH, dW
 
 
 def fused_kl_from_host(dev_bufs: dict, host: dict, T=1.0, chunk=0, workspace=None, out=None):

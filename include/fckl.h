@@ -151,6 +151,34 @@ fckl_status fckl_fwd_bwd(const fckl_problem* prob, const void* hidden, const voi
                          float* dH, float* dW,
                          void* workspace, size_t workspace_bytes, void* stream);
 
+/* Bytes of device workspace fckl_fwd_bwd_host needs: the fckl_workspace_bytes
+ * layout followed by device copies of hidden, topk_idx, topk_logit, row_mask
+ * and the loss.  0 when the problem is invalid. */
+size_t fckl_host_workspace_bytes(const fckl_problem* prob);
+
+/* Forward + backward with the per-step inputs in HOST memory: hidden [N,H]
+ * bf16, topk_idx [N,K], topk_logit [N,K] and row_mask [N] (or NULL) are host
+ * pointers; W stays a device pointer (the student's resident output
+ * projection); dH and dW are device outputs as in fckl_fwd_bwd; the loss is
+ * copied to the host scalar *loss_host at the end of the call's work on
+ * `stream`.  (An addition of this library: the pages feed the loss from
+ * activations already on the GPU and a teacher cache read from storage.)
+ *   - The inputs go to the device in chunk-sized pieces on a copy stream of the
+ *     library's own (one per device, created on first use), so the copy of
+ *     chunk c+1 overlaps the kernels of chunk c; each chunk waits on the
+ *     caller's stream only for its own piece.  With a row mask, the call reads
+ *     the host mask once on the host to place the piece boundaries.
+ *   - Host buffers must stay valid and unchanged until the stream has passed
+ *     the call; page-locked (pinned) memory keeps the copies asynchronous.
+ *   - The device copies live in the workspace (fckl_host_workspace_bytes), so
+ *     the call allocates no device memory.  Calls from several host threads
+ *     are serialised while they enqueue.
+ * Errors as fckl_fwd_bwd; device-side errors come back through fckl_check. */
+fckl_status fckl_fwd_bwd_host(const fckl_problem* prob, const void* hidden_host, const void* W,
+                              const int32_t* topk_idx_host, const float* topk_logit_host,
+                              const uint8_t* row_mask_host, float* loss_host, float* dH, float* dW,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
 /* Forward only (loss and optional row_loss), like fckl_fwd, but without a
  * workspace argument: the call allocates nothing and takes no memory from the
  * caller beyond its inputs and outputs.  It is meant for callers that cannot

@@ -134,3 +134,26 @@ def test_noalloc_rejects_oversized_problem():
     assert fk.fckl_fwd_noalloc(prob, f, f, f, f, None, f, None, None, None) == fk.FCKL_ERR_WORKSPACE
     bad = FcklProblem(64, 60, 512, 8, 1.0, 0)  # H % 8 != 0
     assert fk.fckl_fwd_noalloc(bad, f, f, f, f, None, f, None, None, None) == fk.FCKL_ERR_UNSUPPORTED
+
+
+def test_host_input_entry_point_checks():
+    """The host-input call sizes its workspace as the device-input layout plus
+    device copies of the inputs, and rejects missing host buffers and a short
+    workspace before it touches the device."""
+    p = FcklProblem(300, 64, 700, 9, 1.0, 100)
+    base = fk.fckl_workspace_bytes(p)
+    host = fk.fckl_host_workspace_bytes(p)
+    assert host >= base + 300 * 64 * 2 + 2 * 300 * 9 * 4 + 300 + 4
+    assert host < base + 300 * 64 * 2 + 2 * 300 * 9 * 4 + 300 + 4 + 5 * 256
+    assert fk.fckl_host_workspace_bytes(FcklProblem(300, 64, 700, 0, 1.0, 0)) == 0
+    f = 1 << 20
+    args = [f, f, f, f, None, f, f, f, f, host]
+    for i in (0, 2, 3, 5):
+        a = list(args)
+        a[i] = None
+        assert fk.fckl_fwd_bwd_host(p, *a, None) == fk.FCKL_ERR_INVALID_ARG, i
+    a = list(args)
+    a[9] = host - 1
+    assert fk.fckl_fwd_bwd_host(p, *a, None) == fk.FCKL_ERR_WORKSPACE
+    bad = FcklProblem(300, 60, 700, 9, 1.0, 100)
+    assert fk.fckl_fwd_bwd_host(bad, *args, None) == fk.FCKL_ERR_UNSUPPORTED
