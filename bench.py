@@ -62,6 +62,8 @@ def parse():
     ap.add_argument("--config", type=int, default=1)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="also time the step replayed from a captured CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=0, help="rows in the oracle sample (0 = auto)")
     ap.add_argument("--profile-json", default="")
@@ -299,6 +301,10 @@ def run_cuda(args):
                 "tflops": (p["flops"] / (p["total_ms"] / 1e3) / 1e12) if p["flops"] else None}
                for p in breakdown]
 
+    graph = None
+    if args.graph:
+        graph = measure_graph(torch, dev, step, args.steps, cfg, world)
+
     e2e = None
     if not args.no_e2e:
         e2e = measure_e2e(torch, dev, inp, cfg, ws, args.steps, world, outs)
@@ -325,7 +331,7 @@ def run_cuda(args):
                                  "dense_spec_2250": tflops / world / 2250.0},
                 "peak_mem_gib": peak_gib, "loss": loss_val,
                 "roofline": roofline, "kernels": kernels,
-                "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
+                "cpu_baseline": cpu, "e2e": e2e, "clocks": clk, "graph": graph,
                 "gpu_launches": launches_per_step * args.steps}
         print(json.dumps(line), flush=True)
         if args.profile_json:
@@ -335,6 +341,32 @@ def run_cuda(args):
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def measure_graph(torch, dev, step, steps, cfg, world):
+    """The same step captured once into a CUDA graph and replayed (no per-launch
+    host work); timed like the main region."""
+    s = torch.cuda.Stream(dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(s):
+        step()
+    torch.cuda.current_stream(dev).wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    del g
+    return {"value": cfg.N * world / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms}
 
 
 def measure_e2e(torch, dev, inp, cfg, ws, steps, world, outs):
