@@ -52,7 +52,7 @@ bool supported_problem(const fckl_problem* p) {
 }
 
 long long resolve_chunk(const fckl_problem* p) {
-  const long long Vp = align_up((size_t)p->V, 8);
+  const long long Vp = align_up((size_t)p->V, 64);
   long long C = p->chunk;
   if (C == 0) {
     const long long budget = 512ll << 20;
@@ -68,7 +68,9 @@ long long resolve_chunk(const fckl_problem* p) {
 Layout make_layout(const fckl_problem* p, bool full = true) {
   Layout L{};
   L.N = p->N; L.H = p->H; L.V = p->V; L.K = p->K;
-  L.Vp = (long long)align_up((size_t)p->V, 8);
+  // dlogits rows are padded to a multiple of 64 columns (zeros in the pad), so
+  // the dW GEMM can read them as whole 64-column chunks.
+  L.Vp = (long long)align_up((size_t)p->V, 64);
   L.C = resolve_chunk(p);
   L.nchunks = cdiv(L.N, L.C);
   // The dW GEMM reduces over the rows of its dlogits block, and each launch
@@ -136,6 +138,35 @@ bool make_map(CUtensorMap* m, const void* base, long long inner, long long outer
              const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D view of a row-major bf16 [outer, inner] matrix (inner % 64 == 0) for
+// MN-major operand loads: dims {64, outer, inner / 64}, strides {row pitch,
+// 128 B}; a box {64, box_outer, 2} brings two adjacent 64-wide column chunks,
+// stored chunk after chunk in shared memory exactly as two 2-D boxes would be.
+bool make_map_mn3(CUtensorMap* m, const void* base, long long inner, long long outer,
+                  long long stride_bytes, int box_outer) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (enc == nullptr || inner % 64 != 0) return false;
+  cuuint64_t dims[3] = {64, (cuuint64_t)outer, (cuuint64_t)(inner / 64)};
+  cuuint64_t strides[2] = {(cuuint64_t)stride_bytes, 128};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_outer, 2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// MN-major operand map: the 3-D form when the column count allows it and the
+// driver accepts it (sets *is3d), else the 2-D form with 64-column boxes.
+bool make_map_mn(CUtensorMap* m, const void* base, long long inner, long long outer,
+                 long long stride_bytes, int* is3d) {
+  *is3d = 0;
+  if (inner % 64 == 0 && make_map_mn3(m, base, inner, outer, stride_bytes, BK)) {
+    *is3d = 1;
+    return true;
+  }
+  return make_map(m, base, inner, outer, stride_bytes, 64, BK);
 }
 
 // ---------------------------------------------------------------- device info
@@ -379,7 +410,8 @@ fckl_status run(const Request& q) {
 
   CUtensorMap mapW_k, mapW_mn, mapdW;
   if (!make_map(&mapW_k, q.W, L.H, L.V, L.H * 2, BK, BN / 2)) return FCKL_ERR_CUDA;
-  if (bwd && !make_map(&mapW_mn, q.W, L.H, L.V, L.H * 2, 64, BK)) return FCKL_ERR_CUDA;
+  int w3d = 0;
+  if (bwd && !make_map_mn(&mapW_mn, q.W, L.H, L.V, L.H * 2, &w3d)) return FCKL_ERR_CUDA;
   if (bwd && !make_map(&mapdW, q.dW, L.H, L.V, L.H * 4, 32, 32, true)) return FCKL_ERR_CUDA;
 
   const int pairs = std::max(1, dev->sms / 2);  // CTA pairs that run at once
@@ -442,7 +474,7 @@ fckl_status run(const Request& q) {
     CUtensorMap mapH_k;
     if (!make_map(&mapH_k, h_c, L.H, cap, L.H * 2, BK, CM)) return FCKL_ERR_CUDA;
     // Forward units are vocab-major so that concurrent pairs share W tiles.
-    SchedArgs sa_v{SCHED_VOCAB_MAJOR, (int)NT, (int)KBh, 1, 0, rc};
+    SchedArgs sa_v{SCHED_VOCAB_MAJOR, (int)NT, (int)KBh, 1, 0, rc, 0, 0};
     const int Gv = grid_for(MT * NT);
     const double gemm_flops = 2.0 * nr * (double)L.V * (double)L.H;
 
@@ -494,7 +526,8 @@ fckl_status run(const Request& q) {
     // Backward 1: recompute the tiles and form bf16 dlogits = q - p~.
     EpiDlogits::Params pb{V, K, (int)NT, scale2, lse2, sid, tstart, sp, mask_c};
     CUtensorMap mapD_st;
-    if (!make_map(&mapD_st, dlog_c, L.V, cap, L.Vp * 2, 64, 32)) return FCKL_ERR_CUDA;
+    // The store map spans the padded width: the pad columns receive zeros.
+    if (!make_map(&mapD_st, dlog_c, L.Vp, cap, L.Vp * 2, 64, 32)) return FCKL_ERR_CUDA;
     {
       ProfScope ps(K_BWD, st, gemm_flops, 2.0 * (nr + (double)L.V) * L.H + 2.0 * nr * L.V);
       gemm_pair_kernel<EpiDlogits, false, false>
@@ -509,7 +542,7 @@ fckl_status run(const Request& q) {
     if (!make_map(&mapdH, dH_c, L.H, cap, L.H * 4, 32, 32, true)) return FCKL_ERR_CUDA;
     const long long tiles_h = MT * NTh;
     const int S = choose_split(tiles_h, KBv, pairs);
-    SchedArgs sa_h{SCHED_SPLIT_K, (int)NTh, (int)KBv, S, 0, rc};
+    SchedArgs sa_h{SCHED_SPLIT_K, (int)NTh, (int)KBv, S, 0, rc, 0, w3d};
     EpiDH::Params ph{H, invT, ctl};
     {
       ProfScope ps(K_DH, st, gemm_flops,
@@ -532,10 +565,11 @@ fckl_status run(const Request& q) {
     const int gcap = (int)(row0 + cap - grow0);
     const void* h_g = list ? static_cast<const void*>(hstage)
                            : static_cast<const uint8_t*>(q.hidden) + (size_t)grow0 * L.H * 2;
-    if (!make_map(&mapD_mn, dlog, L.V, gcap, L.Vp * 2, 64, BK)) return FCKL_ERR_CUDA;
-    if (!make_map(&mapH_mn, h_g, L.H, gcap, L.H * 2, 64, BK)) return FCKL_ERR_CUDA;
+    int d3d = 0, h3d = 0;
+    if (!make_map_mn(&mapD_mn, dlog, L.Vp, gcap, L.Vp * 2, &d3d)) return FCKL_ERR_CUDA;
+    if (!make_map_mn(&mapH_mn, h_g, L.H, gcap, L.H * 2, &h3d)) return FCKL_ERR_CUDA;
     const long long tiles_w = cdiv(L.V, PM) * NTh;
-    SchedArgs sa_w{SCHED_TILES, (int)NTh, 0, 1, (int)cdiv(L.V, PM), rows_of(grow0, gcap)};
+    SchedArgs sa_w{SCHED_TILES, (int)NTh, 0, 1, (int)cdiv(L.V, PM), rows_of(grow0, gcap), d3d, h3d};
     EpiDW::Params pw{V, H, invT, g0 > 0 ? 1 : 0, ctl};
     if (compact && g0 == 0) {  // with no valid row no dW launch below writes dW
       ProfScope ps(K_ZERO_DW, st, 0.0, 0.0);

@@ -98,6 +98,9 @@ struct SchedArgs {
   int S;       // split-K factor (SCHED_SPLIT_K)
   int MT;      // row tiles of M (SCHED_TILES: M is the vocabulary)
   RowCount rc; // the launch's rows: M of the first two kinds, K of SCHED_TILES
+  // MN-major operands: 1 = the map is 3-D {64, k, MN/64}, so that one box
+  // brings both 64-wide column chunks of a CTA's half tile; 0 = two 2-D boxes.
+  int a3d, b3d;
 };
 
 // Cluster c of G takes units c, c+G, c+2G, ...  In every order above, the
@@ -235,12 +238,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
           const int k0 = kb * BK;
           if (!A_MN) {
             tma_load_2d_pair(a_dst, &tmA, fb, k0, a_row);
+          } else if (sa.a3d) {
+            tma_load_3d_pair(a_dst, &tmA, fb, 0, k0, a_row >> 6);
           } else {
             tma_load_2d_pair(a_dst, &tmA, fb, a_row, k0);
             tma_load_2d_pair(a_dst + 8192, &tmA, fb, a_row + 64, k0);
           }
           if (!B_MN) {
             tma_load_2d_pair(b_dst, &tmB, fb, k0, b_col);
+          } else if (sa.b3d) {
+            tma_load_3d_pair(b_dst, &tmB, fb, 0, k0, b_col >> 6);
           } else {
             tma_load_2d_pair(b_dst, &tmB, fb, b_col, k0);
             tma_load_2d_pair(b_dst + 8192, &tmB, fb, b_col + 64, k0);
