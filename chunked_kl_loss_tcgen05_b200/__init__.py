@@ -21,7 +21,7 @@ __all__ = [
     "fckl_workspace_bytes", "fckl_resolved_chunk", "fckl_fwd", "fckl_fwd_bwd", "fckl_check",
     "fckl_status_string", "FcklKernelStat", "fckl_profile_begin", "fckl_profile_end",
     "fckl_fwd_noalloc", "fckl_student_entropy", "fckl_select_top_rows", "fckl_fwd_bwd_rows",
-    "fckl_host_workspace_bytes", "fckl_fwd_bwd_host",
+    "fckl_host_workspace_bytes", "fckl_fwd_bwd_host", "fckl_fwd_bwd_sliced",
 ]
 
 FCKL_OK = 0
@@ -40,7 +40,8 @@ _LIB = None
 exported_symbols = ("fckl_workspace_bytes", "fckl_resolved_chunk", "fckl_fwd", "fckl_fwd_bwd",
                     "fckl_check", "fckl_status_string", "fckl_profile_begin", "fckl_profile_end",
                     "fckl_fwd_noalloc", "fckl_student_entropy", "fckl_select_top_rows",
-                    "fckl_fwd_bwd_rows", "fckl_host_workspace_bytes", "fckl_fwd_bwd_host")
+                    "fckl_fwd_bwd_rows", "fckl_host_workspace_bytes", "fckl_fwd_bwd_host",
+                    "fckl_fwd_bwd_sliced")
 
 
 FCKL_TEACHER_LOGITS = 0
@@ -95,6 +96,10 @@ def load() -> ctypes.CDLL:
     lib.fckl_fwd.restype = ctypes.c_int
     lib.fckl_fwd_bwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.fckl_fwd_bwd.restype = ctypes.c_int
+    lib.fckl_fwd_bwd_sliced.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp,
+                                         ctypes.c_int32, ctypes.POINTER(vp),
+                                         ctypes.POINTER(ctypes.c_int64)]
+    lib.fckl_fwd_bwd_sliced.restype = ctypes.c_int
     lib.fckl_host_workspace_bytes.argtypes = [P]
     lib.fckl_host_workspace_bytes.restype = sz
     lib.fckl_fwd_bwd_host.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
@@ -163,6 +168,22 @@ def fckl_fwd_bwd_host(prob, hidden_host, W, topk_idx_host, topk_logit_host, row_
                                         _ptr(row_mask_host), _ptr(loss_host), _ptr(dH), _ptr(dW),
                                         _ptr(workspace), ctypes.c_size_t(int(workspace_bytes)),
                                         _ptr(stream)))
+
+
+def fckl_fwd_bwd_sliced(prob, hidden, W, topk_idx, topk_logit, row_mask, loss, row_loss, dH, dW,
+                        workspace, workspace_bytes, stream, events) -> tuple:
+    """fckl_fwd_bwd with the last dW launch split into len(events) vocabulary
+    slices; events are cudaEvent_t handles (ints).  Returns (status, row
+    boundaries of the slices as a list of len(events) + 1 ints)."""
+    n = len(events)
+    ev = (ctypes.c_void_p * max(n, 1))(*[ctypes.c_void_p(int(e)) if e else None for e in events])
+    rows = (ctypes.c_int64 * (n + 1))()
+    st = load().fckl_fwd_bwd_sliced(ctypes.byref(prob), _ptr(hidden), _ptr(W), _ptr(topk_idx),
+                                    _ptr(topk_logit), _ptr(row_mask), _ptr(loss), _ptr(row_loss),
+                                    _ptr(dH), _ptr(dW), _ptr(workspace),
+                                    ctypes.c_size_t(int(workspace_bytes)), _ptr(stream),
+                                    ctypes.c_int32(n), ev, rows)
+    return int(st), list(rows)
 
 
 def fckl_fwd_noalloc(prob, hidden, W, topk_idx, topk_logit, row_mask, loss, row_loss,

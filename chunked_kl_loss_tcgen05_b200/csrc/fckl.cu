@@ -313,6 +313,12 @@ struct Request {
   // Host-input calls: ready[0] marks the row mask copied to the device,
   // ready[1 + c] the rows chunk c reads; the chunk waits for it on the stream.
   const cudaEvent_t* ready = nullptr;
+  // Sliced dW: the last dW launch runs as n_slices launches over consecutive
+  // vocabulary ranges; slice_events[i] is recorded after slice i and
+  // slice_rows[i..i+1] receives its dW row range.
+  int n_slices = 0;
+  cudaEvent_t const* slice_events = nullptr;
+  int64_t* slice_rows = nullptr;
 };
 
 fckl_status run(const Request& q) {
@@ -568,24 +574,44 @@ fckl_status run(const Request& q) {
     int d3d = 0, h3d = 0;
     if (!make_map_mn(&mapD_mn, dlog, L.Vp, gcap, L.Vp * 2, &d3d)) return FCKL_ERR_CUDA;
     if (!make_map_mn(&mapH_mn, h_g, L.H, gcap, L.H * 2, &h3d)) return FCKL_ERR_CUDA;
-    const long long tiles_w = cdiv(L.V, PM) * NTh;
-    SchedArgs sa_w{SCHED_TILES, (int)NTh, 0, 1, (int)cdiv(L.V, PM), rows_of(grow0, gcap), d3d, h3d};
+    const long long MTv = cdiv(L.V, PM);
     EpiDW::Params pw{V, H, invT, g0 > 0 ? 1 : 0, ctl};
     if (compact && g0 == 0) {  // with no valid row no dW launch below writes dW
       ProfScope ps(K_ZERO_DW, st, 0.0, 0.0);
       k_zero_if_no_valid<<<2 * pairs, 256, 0, st>>>(reinterpret_cast<float4*>(q.dW),
                                                      L.V * L.H / 4, ctl);
     }
-    {
-      const double gr = prof_rows < 0
-                            ? (double)gcap
-                            : (double)std::max(0LL, std::min<long long>(gcap, prof_rows - grow0));
-      ProfScope ps(K_DW, st, 2.0 * gr * (double)L.V * (double)L.H,
-                   2.0 * gr * (double)L.V + 2.0 * gr * L.H +
-                       (g0 > 0 ? 8.0 : 4.0) * (double)L.V * L.H);
-      gemm_pair_kernel<EpiDW, true, true>
-          <<<grid_for(tiles_w), GEMM_THREADS, pair_smem_bytes<EpiDW>(), st>>>(
-              mapD_mn, mapH_mn, mapdW, pw, sa_w, ca);
+    // One launch over all vocabulary tiles, or -- for the last group of a
+    // sliced call -- one launch per slice, each followed by its event.
+    const bool sliced = q.n_slices > 0 && c + 1 == nchunks;
+    const long long ns = sliced ? std::min<long long>(q.n_slices, MTv) : 1;
+    const double gr = prof_rows < 0
+                          ? (double)gcap
+                          : (double)std::max(0LL, std::min<long long>(gcap, prof_rows - grow0));
+    for (long long i = 0; i < ns; ++i) {
+      const long long mt0 = i * MTv / ns, mt1 = (i + 1) * MTv / ns;
+      const long long v0 = mt0 * PM, v1 = std::min<long long>(L.V, mt1 * PM);
+      SchedArgs sa_w{SCHED_TILES, (int)NTh, 0, 1, (int)(mt1 - mt0), rows_of(grow0, gcap), d3d, h3d,
+                     (int)mt0};
+      {
+        const double vs = (double)(v1 - v0);
+        ProfScope ps(K_DW, st, 2.0 * gr * vs * (double)L.H,
+                     2.0 * gr * vs + 2.0 * gr * L.H * ns + (g0 > 0 ? 8.0 : 4.0) * vs * L.H);
+        gemm_pair_kernel<EpiDW, true, true>
+            <<<grid_for((mt1 - mt0) * NTh), GEMM_THREADS, pair_smem_bytes<EpiDW>(), st>>>(
+                mapD_mn, mapH_mn, mapdW, pw, sa_w, ca);
+      }
+      if (sliced) {
+        if (cudaEventRecord(q.slice_events[i], st) != cudaSuccess) return FCKL_ERR_CUDA;
+        q.slice_rows[i] = v0;
+        q.slice_rows[i + 1] = v1;
+      }
+    }
+    if (sliced) {  // slices beyond the vocabulary tiles are empty
+      for (long long i = ns; i < q.n_slices; ++i) {
+        if (cudaEventRecord(q.slice_events[i], st) != cudaSuccess) return FCKL_ERR_CUDA;
+        q.slice_rows[i + 1] = L.V;
+      }
     }
   }
   if (!ent) {
@@ -749,6 +775,28 @@ fckl_status fckl_fwd_bwd(const fckl_problem* prob, const void* hidden, const voi
   q.prob = prob; q.hidden = hidden; q.W = W; q.topk_idx = topk_idx; q.topk_logit = topk_logit;
   q.row_mask = row_mask; q.loss = loss; q.row_loss = row_loss; q.dH = dH; q.dW = dW;
   q.workspace = workspace; q.ws_bytes = workspace_bytes; q.stream = stream;
+  return run(q);
+}
+
+fckl_status fckl_fwd_bwd_sliced(const fckl_problem* prob, const void* hidden, const void* W,
+                                const int32_t* topk_idx, const float* topk_logit,
+                                const uint8_t* row_mask, float* loss, float* row_loss, float* dH,
+                                float* dW, void* workspace, size_t workspace_bytes, void* stream,
+                                int32_t n_slices, void* const* slice_events,
+                                int64_t* slice_rows) {
+  if (n_slices < 1 || n_slices > 4096 || slice_events == nullptr || slice_rows == nullptr)
+    return FCKL_ERR_INVALID_ARG;
+  for (int32_t i = 0; i < n_slices; ++i)
+    if (slice_events[i] == nullptr) return FCKL_ERR_INVALID_ARG;
+  Request q;
+  q.mode = Mode::kFwdBwd;
+  q.prob = prob; q.hidden = hidden; q.W = W; q.topk_idx = topk_idx; q.topk_logit = topk_logit;
+  q.row_mask = row_mask; q.loss = loss; q.row_loss = row_loss; q.dH = dH; q.dW = dW;
+  q.workspace = workspace; q.ws_bytes = workspace_bytes; q.stream = stream;
+  q.n_slices = n_slices;
+  q.slice_events = reinterpret_cast<cudaEvent_t const*>(slice_events);
+  q.slice_rows = slice_rows;
+  slice_rows[0] = 0;
   return run(q);
 }
 

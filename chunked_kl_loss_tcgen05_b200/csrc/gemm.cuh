@@ -101,6 +101,7 @@ struct SchedArgs {
   // MN-major operands: 1 = the map is 3-D {64, k, MN/64}, so that one box
   // brings both 64-wide column chunks of a CTA's half tile; 0 = two 2-D boxes.
   int a3d, b3d;
+  int mt0;     // SCHED_TILES: first row tile of the launch (launches over a slice of M)
 };
 
 // Cluster c of G takes units c, c+G, c+2G, ...  In every order above, the
@@ -136,8 +137,9 @@ struct PairSched {
       w.kb0 = (int)((long long)ks * KB / a.S);
       w.kb1 = (int)((long long)(ks + 1) * KB / a.S);
     } else {
-      w.mt = (int)(u / a.NT);
-      w.nt = (int)(u - (long long)w.mt * a.NT);
+      const int t = (int)(u / a.NT);
+      w.nt = (int)(u - (long long)t * a.NT);
+      w.mt = a.mt0 + t;
       w.kb0 = 0; w.kb1 = KB;
     }
     w.rows = rows;

@@ -11,11 +11,13 @@ from __future__ import annotations
 import torch
 
 from . import (FcklError, FcklProblem, FCKL_OK, fckl_check, fckl_fwd, fckl_fwd_bwd,
-               fckl_fwd_bwd_host, fckl_host_workspace_bytes, fckl_workspace_bytes)
+               fckl_fwd_bwd_host, fckl_fwd_bwd_sliced, fckl_host_workspace_bytes,
+               fckl_workspace_bytes)
 
 __all__ = ["make_problem", "alloc_workspace", "fused_kl_fwd", "fused_kl_fwd_bwd", "student_entropy",
            "select_top_rows", "fused_kl_rows", "arrays_to_device",
            "fused_kl_from_host", "alloc_host_workspace", "fused_kl_fwd_bwd_host",
+           "fused_kl_fwd_bwd_sliced",
            "FusedChunkedKL", "fused_chunked_kl_loss"]
 
 
@@ -90,6 +92,39 @@ def fused_kl_fwd_bwd(hidden, W, topk_idx, topk_logit, row_mask=None, T=1.0, chun
         if st != FCKL_OK:
             raise FcklError(st, "fckl_check")
     return loss, row_loss, dH, dW
+
+
+def fused_kl_fwd_bwd_sliced(hidden, W, topk_idx, topk_logit, row_mask=None, T=1.0, chunk=0,
+                            workspace=None, n_slices=4, teacher=0, n_valid_total=0, out=None):
+    """fused_kl_fwd_bwd whose last dW launch is split into ``n_slices``
+    vocabulary slices.  Returns (loss[1], dH, dW, slices) with slices a list of
+    (row0, row1, event): dW[row0:row1] is final once ``event`` (a
+    torch.cuda.Event recorded on the current stream) has completed."""
+    hidden, W = _bits(hidden), _bits(W)
+    _check_inputs(hidden, W, topk_idx, topk_logit, row_mask)
+    prob = make_problem(hidden, W, topk_idx, T, chunk, teacher, n_valid_total)
+    dev = hidden.device
+    if workspace is None:
+        workspace = alloc_workspace(prob, dev)
+    if out is None:
+        out = (torch.empty(1, dtype=torch.float32, device=dev),
+               torch.empty(prob.N, prob.H, dtype=torch.float32, device=dev),
+               torch.empty(prob.V, prob.H, dtype=torch.float32, device=dev))
+    loss, dH, dW = out
+    stream = torch.cuda.current_stream(dev)
+    events = [torch.cuda.Event() for _ in range(n_slices)]
+    for e in events:
+        e.record(stream)  # creates the CUDA event; the call records it again
+    st, rows = fckl_fwd_bwd_sliced(prob, hidden.data_ptr(), W.data_ptr(), topk_idx.data_ptr(),
+                                   topk_logit.data_ptr(),
+                                   None if row_mask is None else row_mask.data_ptr(),
+                                   loss.data_ptr(), None, dH.data_ptr(), dW.data_ptr(),
+                                   workspace.data_ptr(), workspace.numel(), stream.cuda_stream,
+                                   [e.cuda_event for e in events])
+    if st != FCKL_OK:
+        raise FcklError(st, "fckl_fwd_bwd_sliced")
+    slices = [(rows[i], rows[i + 1], events[i]) for i in range(n_slices)]
+    return loss, dH, dW, slices
 
 
 def fused_kl_fwd(hidden, W, topk_idx, topk_logit, row_mask=None, T=1.0, chunk=0,

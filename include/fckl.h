@@ -151,6 +151,27 @@ fckl_status fckl_fwd_bwd(const fckl_problem* prob, const void* hidden, const voi
                          float* dH, float* dW,
                          void* workspace, size_t workspace_bytes, void* stream);
 
+/* fckl_fwd_bwd with the dW write-out exposed slice by slice, so that a caller
+ * can reduce finished parts of dW across ranks while the rest is computed
+ * (row-sharded data parallelism: the dW all-reduce overlaps the last dW GEMM).
+ * The last dW launch runs as min(n_slices, ceil(V/256)) launches over
+ * consecutive vocabulary ranges; after the launch that finishes dW rows
+ * [slice_rows[i], slice_rows[i+1]) the call records slice_events[i] (a
+ * cudaEvent_t of the caller, on the current device) on `stream`.  Slices past
+ * the vocabulary tiles are empty (their event is recorded after the last one).
+ * slice_rows (host, n_slices + 1 entries) is filled before the call returns;
+ * slice_rows[0] = 0 and slice_rows[n_slices] = V.  The dW rows of slice i are
+ * final once event i has fired; everything else (loss, dH) is as in
+ * fckl_fwd_bwd, complete in stream order after the call's work.
+ * 1 <= n_slices <= 4096, every event non-NULL, else FCKL_ERR_INVALID_ARG.
+ * (An addition of this library for multi-GPU use; the pages run on one GPU.) */
+fckl_status fckl_fwd_bwd_sliced(const fckl_problem* prob, const void* hidden, const void* W,
+                                const int32_t* topk_idx, const float* topk_logit,
+                                const uint8_t* row_mask, float* loss, float* row_loss, float* dH,
+                                float* dW, void* workspace, size_t workspace_bytes, void* stream,
+                                int32_t n_slices, void* const* slice_events,
+                                int64_t* slice_rows);
+
 /* Bytes of device workspace fckl_fwd_bwd_host needs: the fckl_workspace_bytes
  * layout followed by device copies of hidden, topk_idx, topk_logit, row_mask
  * and the loss.  0 when the problem is invalid. */

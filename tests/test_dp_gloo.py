@@ -42,7 +42,10 @@ def _worker(rank, world, port, case, out_q):
                                         mask.numpy(), T, n_valid=n_valid_total)
             loss = torch.tensor([o["row_loss"].sum() / n_valid_total if n_valid_total else 0.0],
                                 dtype=torch.float64)
-            return loss, None, torch.from_numpy(o["dH"]), torch.from_numpy(o["dW"])
+            V = ww.shape[0]
+            cuts = [0, V // 3, V // 3, V]  # uneven slices, one of them empty
+            slices = [(cuts[i], cuts[i + 1], None) for i in range(3)]
+            return loss, torch.from_numpy(o["dH"]), torch.from_numpy(o["dW"]), slices
 
         loss, dH, dW = fused_kl_fwd_bwd_dp(
             h, Wd, torch.from_numpy(inp.topk_idx[lo:hi]), torch.from_numpy(inp.topk_logit[lo:hi]),

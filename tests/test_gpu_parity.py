@@ -291,6 +291,28 @@ def test_global_valid_count_scales_loss_and_grads():
     assert abs(l2.item() - o2["row_loss"].sum() / (2 * nv)) <= LOSS_RTOL * abs(o["loss"] / 2)
 
 
+@pytest.mark.parametrize("n_slices", [1, 3, 7, 40])
+def test_sliced_dw_matches_plain_call(n_slices):
+    """Splitting the last dW launch into vocabulary slices changes nothing but
+    the launch pattern; the slices cover dW's rows in order and every event
+    has fired once the stream is done.  V = 2000 has 8 tiles of 256, so 40
+    slices leave 32 empty ones."""
+    from chunked_kl_loss_tcgen05_b200.torch_api import fused_kl_fwd_bwd_sliced
+    inp = synth.make_custom(600, 128, 2000, 10, mask_frac=0.1, seed=83, chunk=128)
+    d = arrays_to_device(inp.hidden, inp.W, inp.topk_idx, inp.topk_logit, inp.row_mask)
+    l1, _, dH1, dW1 = fused_kl_fwd_bwd(*d, chunk=128)
+    l2, dH2, dW2, slices = fused_kl_fwd_bwd_sliced(*d, chunk=128, n_slices=n_slices)
+    torch.cuda.synchronize()
+    assert l2.item() == l1.item()
+    assert torch.equal(dW2, dW1)
+    assert rel_fro(dH2.cpu().numpy(), dH1.cpu().numpy()) < 1e-6
+    bounds = [0] + [r1 for _, r1, _ in slices]
+    assert [r0 for r0, _, _ in slices] == bounds[:-1] and bounds[-1] == 2000
+    assert all(r0 % 256 == 0 for r0, r1, _ in slices if r1 > r0)
+    assert sum(r1 > r0 for r0, r1, _ in slices) == min(n_slices, 8)
+    assert all(ev.query() for _, _, ev in slices)
+
+
 def test_dp_wrapper_single_rank_nccl():
     """The data-parallel wrapper on one NCCL rank equals the plain call."""
     import torch.distributed as dist
