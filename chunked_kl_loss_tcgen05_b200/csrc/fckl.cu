@@ -425,6 +425,9 @@ fckl_status run(const Request& q) {
   const long long KBh = cdiv(L.H, BK);
   const long long NTh = cdiv(L.H, BN);
   const long long KBv = cdiv(L.V, BK);
+  // dH and dW tile the hidden dimension by 256; a last tile of at most 128
+  // columns (e.g. H = 2880) runs as a half-width MMA.
+  const int narrow_h = (L.H % BN != 0 && L.H % BN <= 128) ? 1 : 0;
   const long long R = user_list ? q.n_rows : L.N;  // rows (or list entries), upper bound
   const long long nchunks = cdiv(R, L.C);
   const long long G = std::min<long long>(nchunks, L.G);
@@ -548,7 +551,7 @@ fckl_status run(const Request& q) {
     if (!make_map(&mapdH, dH_c, L.H, cap, L.H * 4, 32, 32, true)) return FCKL_ERR_CUDA;
     const long long tiles_h = MT * NTh;
     const int S = choose_split(tiles_h, KBv, pairs);
-    SchedArgs sa_h{SCHED_SPLIT_K, (int)NTh, (int)KBv, S, 0, rc, 0, w3d};
+    SchedArgs sa_h{SCHED_SPLIT_K, (int)NTh, (int)KBv, S, 0, rc, 0, w3d, 0, narrow_h};
     EpiDH::Params ph{H, invT, ctl};
     {
       ProfScope ps(K_DH, st, gemm_flops,
@@ -592,7 +595,7 @@ fckl_status run(const Request& q) {
       const long long mt0 = i * MTv / ns, mt1 = (i + 1) * MTv / ns;
       const long long v0 = mt0 * PM, v1 = std::min<long long>(L.V, mt1 * PM);
       SchedArgs sa_w{SCHED_TILES, (int)NTh, 0, 1, (int)(mt1 - mt0), rows_of(grow0, gcap), d3d, h3d,
-                     (int)mt0};
+                     (int)mt0, narrow_h};
       {
         const double vs = (double)(v1 - v0);
         ProfScope ps(K_DW, st, 2.0 * gr * vs * (double)L.H,

@@ -102,7 +102,14 @@ struct SchedArgs {
   // brings both 64-wide column chunks of a CTA's half tile; 0 = two 2-D boxes.
   int a3d, b3d;
   int mt0;     // SCHED_TILES: first row tile of the launch (launches over a slice of M)
+  // 1: the last column tile holds at most 128 columns, so it runs as an
+  // N = 128 MMA (each CTA of the pair stages 64 columns of B) instead of 256.
+  int narrow_tail;
 };
+
+__device__ __forceinline__ bool narrow_unit(const SchedArgs& a, const Work& w) {
+  return a.narrow_tail && w.nt == a.NT - 1;
+}
 
 // Cluster c of G takes units c, c+G, c+2G, ...  In every order above, the
 // clusters running at the same moment touch a narrow band of the streamed
@@ -222,7 +229,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       bool ok = true;
       while (ok && sch.next(w)) {
         const int a_row = w.mt * PM + (int)rank * CM;
-        const int b_col = w.nt * BN + (int)rank * (BN / 2);
+        const int b_col = w.nt * BN + (int)rank * (narrow_unit(sa, w) ? 64 : BN / 2);
         for (int kb = w.kb0; kb < w.kb1; ++kb) {
           if (!wait_phase(smem_u32(&empty[stage]), phase ^ 1u, wc, SITE_PROD_EMPTY)) {
             ok = false;
@@ -277,13 +284,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
-      constexpr uint32_t idesc = idesc_bf16_f32(PM, BN, A_MN, B_MN);
+      constexpr uint32_t idesc_full = idesc_bf16_f32(PM, BN, A_MN, B_MN);
+      constexpr uint32_t idesc_narrow = idesc_bf16_f32(PM, 128, A_MN, B_MN);
       bool ok = true;
       int skip = ca.debug_skip_commit;
       while (ok && sch.next(w)) {
         if (!wait_phase(smem_u32(&tempty[acc]), acc_phase ^ 1u, wc, SITE_MMA_TEMPTY)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        const uint32_t idesc = narrow_unit(sa, w) ? idesc_narrow : idesc_full;
         for (int kb = w.kb0; kb < w.kb1; ++kb) {
           if (!wait_phase(smem_u32(&full[stage]), phase, wc, SITE_MMA_FULL)) {
             ok = false;
