@@ -55,7 +55,10 @@ long long resolve_chunk(const fckl_problem* p) {
   const long long Vp = align_up((size_t)p->V, 64);
   long long C = p->chunk;
   if (C == 0) {
-    const long long budget = 512ll << 20;
+    // 1 GiB: the dW GEMM reduces over >= 4096 rows of dlogits anyway, so at
+    // V = 128K a 4096-row chunk costs no more workspace than smaller chunks
+    // grouped for dW, and halves the launches (and their tail waves).
+    const long long budget = 1024ll << 20;
     C = budget / (Vp * 2) / 128 * 128;
     C = std::max(C, 128ll);
     C = std::min(C, (long long)align_up((size_t)p->N, 64));

@@ -342,7 +342,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     Epi::init(ep, st, sEpi + quarter * (Epi::kSmemBytes / 4), lane);
     while (sch.next(w)) {
       bool ok = true;
-      if (lane == 0) ok = wait_phase(smem_u32(&tfull[acc]), acc_phase, wc, SITE_EPI_TFULL);
+      // A tile's main loop lasts tens of microseconds: the epilogue polls its
+      // accumulator-ready barrier every 2 us (measured ~0.5-0.9% faster steps
+      // under the power cap than polling back to back).
+      if (lane == 0) ok = wait_phase(smem_u32(&tfull[acc]), acc_phase, wc, SITE_EPI_TFULL, 2000);
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (!ok) break;
       tc_fence_after();

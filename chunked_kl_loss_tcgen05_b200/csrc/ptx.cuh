@@ -76,13 +76,16 @@ __device__ __forceinline__ void raise_timeout(const WaitCtx& w, uint32_t site) {
 
 // Waits for completion of the phase with parity `parity`.  Returns false (and
 // raises the abort flag) when the budget runs out, or when another role of the
-// CTA has already aborted.  Never spins without limit.
+// CTA has already aborted.  Never spins without limit.  sleep_ns > 0: sleep
+// between polls (for waits that last many microseconds and can afford the
+// extra latency; fewer issued polls save power under the power cap).
 __device__ __noinline__ bool wait_phase_slow(uint32_t bar, uint32_t parity, const WaitCtx& w,
-                                             uint32_t site) {
+                                             uint32_t site, uint32_t sleep_ns) {
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*w.abort_flag) return false;
+    if (sleep_ns) __nanosleep(sleep_ns);
     if ((it & 15u) == 0u) {
       if (globaltimer_ns() - t0 > w.timeout_ns || it > (1u << 30)) {
         raise_timeout(w, site);
@@ -95,9 +98,9 @@ __device__ __noinline__ bool wait_phase_slow(uint32_t bar, uint32_t parity, cons
 // The common case -- the phase has already completed -- stays inline; the
 // bounded loop is a call.
 __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, const WaitCtx& w,
-                                           uint32_t site) {
+                                           uint32_t site, uint32_t sleep_ns = 0) {
   if (mbar_try_wait(bar, parity)) return true;
-  return wait_phase_slow(bar, parity, w, site);
+  return wait_phase_slow(bar, parity, w, site, sleep_ns);
 }
 
 // Cleanup wait: ignores the abort flag (it is used to let in-flight copies and

@@ -82,7 +82,7 @@ typedef enum {
 } fckl_status;
 
 /* Problem description.  chunk = rows per chunk (0 = automatic: the largest
- * multiple of 128 rows whose bf16 dlogits block [chunk, V] fits in 512 MiB,
+ * multiple of 128 rows whose bf16 dlogits block [chunk, V] fits in 1 GiB,
  * capped at N rounded up to 64).  The dW GEMM runs once per group of
  * ceil(4096 / chunk) consecutive chunks (at most all of them), so that each
  * read-modify-write of dW covers at least 4096 rows; the workspace holds that

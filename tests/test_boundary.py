@@ -47,16 +47,16 @@ def test_status_strings():
 
 def test_workspace_and_chunk_rules():
     p1 = FcklProblem(8192, 3072, 128256, 100, 1.0, 0)
-    assert fk.fckl_resolved_chunk(p1) == 2048          # 512 MiB of bf16 dlogits
+    assert fk.fckl_resolved_chunk(p1) == 4096          # 1 GiB of bf16 dlogits
     p3 = FcklProblem(131072, 2880, 201088, 100, 1.0, 0)
-    assert fk.fckl_resolved_chunk(p3) == 1280
+    assert fk.fckl_resolved_chunk(p3) == 2560
     p0 = FcklProblem(256, 256, 4096, 16, 1.0, 64)
     assert fk.fckl_resolved_chunk(p0) == 64
     assert fk.fckl_resolved_chunk(FcklProblem(100, 256, 4096, 16, 1.0, 0)) == 100
     assert fk.fckl_resolved_chunk(FcklProblem(100, 256, 4096, 16, 1.0, 4096)) == 100
     # workspace holds the chunk's bf16 dlogits block and is linear in N beyond it
     w = fk.fckl_workspace_bytes(p1)
-    assert w >= 2048 * 128256 * 2
+    assert w >= 4096 * 128256 * 2
     a = fk.fckl_workspace_bytes(FcklProblem(32768, 4096, 128256, 100, 1.0, 1024))
     b = fk.fckl_workspace_bytes(FcklProblem(65536, 4096, 128256, 100, 1.0, 1024))
     assert b - a == 32768 * 8    # only the per-row loss and the compacted row list grow
