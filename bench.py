@@ -84,6 +84,12 @@ def workload_config(cfg: synth.Config, C: int) -> dict:
             "data": "synthetic seeded (synth recipe)"}
 
 
+def resolved_chunk(cfg: synth.Config) -> int:
+    """The chunk the library uses for this workload (host arithmetic only)."""
+    from chunked_kl_loss_tcgen05_b200 import FcklProblem, fckl_resolved_chunk
+    return fckl_resolved_chunk(FcklProblem(cfg.N, cfg.H, cfg.V, cfg.K, cfg.T, cfg.chunk))
+
+
 # ------------------------------------------------------------------ oracle arm
 def oracle_rows_per_sec(inp, n_rows, reps=1):
     import oracle
@@ -127,7 +133,8 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": workload_config(cfg, 0),
+            "config": dict(workload_config(cfg, resolved_chunk(cfg)),
+                           parallelism=f"replicas{world}", flush="inputs larger than L2"),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_cores(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
