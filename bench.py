@@ -350,6 +350,16 @@ def run_cuda(args):
     return 0
 
 
+def max_over_ranks(torch, dev, ms, world):
+    """The slowest rank's time (every rank calls this at the same point)."""
+    if world == 1:
+        return ms
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def measure_graph(torch, dev, step, steps, cfg, world):
     """The same step captured once into a CUDA graph and replayed (no per-launch
     host work); timed like the main region."""
@@ -371,7 +381,7 @@ def measure_graph(torch, dev, step, steps, cfg, world):
         g.replay()
     e1.record(stream)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / steps
+    ms = max_over_ranks(torch, dev, e0.elapsed_time(e1) / steps, world)
     del g
     return {"value": cfg.N * world / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms}
 
@@ -409,7 +419,7 @@ def measure_e2e(torch, dev, inp, cfg, ws, steps, world, outs):
         call()  # returns after the loss has reached the host
     e1.record(stream)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / steps
+    ms = max_over_ranks(torch, dev, e0.elapsed_time(e1) / steps, world)
     del hws, W
     return {"value": cfg.N * world / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": 4, "steps": steps,
