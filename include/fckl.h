@@ -34,9 +34,11 @@
  *   T^2 factor (the gradients are those of `loss` itself, upstream grad 1).
  *
  * Common conventions for every entry point:
- *   - All array pointers are DEVICE pointers into memory the caller owns; the
- *     library allocates nothing (device or host) and keeps no state between
- *     calls except a per-device cache of kernel attributes.
+ *   - Array pointers are DEVICE pointers into memory the caller owns (except
+ *     the host inputs of fckl_fwd_bwd_host).  The library allocates no device
+ *     memory; between calls it keeps only a per-device cache of kernel
+ *     attributes, the copy stream and events of fckl_fwd_bwd_host, the
+ *     profiler's events and the static scratch of fckl_fwd_noalloc.
  *   - Arrays are dense and row-major.  hidden, W, dH and dW must start on a
  *     16-byte boundary (TMA), the others on a 4-byte boundary:
  *       hidden     bf16  [N, H]      (raw bfloat16 bit patterns)
