@@ -70,6 +70,10 @@ def parse():
     ap.add_argument("--profile-json", default="")
     ap.add_argument("--mem-sweep", action="store_true",
                     help="print peak device memory vs sequence length instead of timing")
+    ap.add_argument("--vs-cublas", type=float, default=0.0, metavar="SECONDS",
+                    help="instead of the contract line: run the fused step and the four plain "
+                         "cuBLAS GEMMs of the same shapes back to back for SECONDS each, clocks "
+                         "sampled, and print both")
     return ap.parse_args()
 
 
@@ -462,12 +466,84 @@ def run_mem_sweep(args):
     return 0
 
 
+def run_vs_cublas(args):
+    """Same-conditions comparison: the fused forward+backward step against the
+    four plain cuBLAS bf16 GEMMs of the same shapes (logits, their recompute,
+    dH, dW; no loss arithmetic, bf16 outputs), each run back to back for the
+    same time with clocks and power sampled, so that both see the same power
+    cap.  A measurement aid, not part of the contract line."""
+    import torch
+    from chunked_kl_loss_tcgen05_b200 import FcklProblem, fckl_resolved_chunk
+    from chunked_kl_loss_tcgen05_b200.torch_api import (alloc_workspace, arrays_to_device,
+                                                        fused_kl_fwd_bwd)
+    torch.cuda.set_device(0)
+    cfg = synth.CONFIGS[args.config]
+    inp = synth.make_inputs(cfg)
+    d = arrays_to_device(inp.hidden, inp.W, inp.topk_idx, inp.topk_logit, inp.row_mask)
+    prob = FcklProblem(cfg.N, cfg.H, cfg.V, cfg.K, cfg.T, cfg.chunk)
+    C = fckl_resolved_chunk(prob)
+    ws = alloc_workspace(prob, d[0].device)
+    outs = (torch.empty(1, device="cuda"), torch.empty(cfg.N, cfg.H, device="cuda"),
+            torch.empty(cfg.V, cfg.H, device="cuda"))
+    n_valid = int(inp.row_mask.sum())
+
+    def fused():
+        fused_kl_fwd_bwd(*d, T=cfg.T, chunk=cfg.chunk, workspace=ws, check=False, out=outs)
+
+    h = d[0][:C].contiguous()
+    W = d[1]
+    g = torch.Generator(device="cuda").manual_seed(7)
+    dl = torch.randn(C, cfg.V, device="cuda", dtype=torch.bfloat16, generator=g)
+    pieces = -(-n_valid // C)
+
+    def gemms():
+        for _ in range(pieces):
+            h @ W.t()
+            h @ W.t()
+            dl @ W
+            dl.t() @ h
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        clocks = ClockSampler(0)
+        clocks.start()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0 = time.time()
+        n = 0
+        e0.record()
+        while time.time() - t0 < args.vs_cublas:
+            fn()
+            n += 1
+            if n % 4 == 0:
+                torch.cuda.synchronize()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n, n, clocks.stop()
+
+    ms_f, n_f, clk_f = timed(fused)
+    ms_c, n_c, clk_c = timed(gemms)
+    fl_f = 8.0 * cfg.H * cfg.V * n_valid
+    fl_c = 4 * 2.0 * C * cfg.V * cfg.H * pieces
+    line = {"workload": cfg.name, "chunk": C,
+            "fused": {"ms_per_step": ms_f, "tflops": fl_f / ms_f / 1e9, "steps": n_f, "clocks": clk_f,
+                      "rows": n_valid},
+            "cublas_4_gemms": {"ms_per_step": ms_c, "tflops": fl_c / ms_c / 1e9, "steps": n_c,
+                               "clocks": clk_c, "rows": C * pieces},
+            "fused_over_cublas_tflops": (fl_f / ms_f) / (fl_c / ms_c)}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
     if args.mem_sweep:
         return run_mem_sweep(args)
+    if args.vs_cublas > 0:
+        return run_vs_cublas(args)
     return run_cuda(args)
 
 
