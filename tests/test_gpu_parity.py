@@ -333,3 +333,26 @@ def test_dp_wrapper_single_rank_nccl():
         assert rel_fro(dH2.cpu().numpy(), dH1.cpu().numpy()) < 1e-6
     finally:
         dist.destroy_process_group()
+
+
+def test_autograd_wrapper_gradients():
+    """loss = fused_chunked_kl_loss(...); (3 * loss).backward() gives hidden.grad
+    and W.grad = 3 * (dH, dW) of the fused call, in the inputs' dtype, and the
+    gradients match the oracle."""
+    from chunked_kl_loss_tcgen05_b200.torch_api import fused_chunked_kl_loss
+    inp = synth.make_custom(300, 128, 2000, 10, T=1.5, mask_frac=0.2, seed=91, chunk=128)
+    d = arrays_to_device(inp.hidden, inp.W, inp.topk_idx, inp.topk_logit, inp.row_mask)
+    h = d[0].view(torch.bfloat16).clone().requires_grad_(True)
+    W = d[1].view(torch.bfloat16).clone().requires_grad_(True)
+    loss = fused_chunked_kl_loss(h, W, d[2], d[3], d[4], T=1.5, chunk=128)
+    (3.0 * loss).backward()
+    l0, _, dH, dW = fused_kl_fwd_bwd(*d, T=1.5, chunk=128)
+    assert loss.item() == l0.item()
+    assert h.grad.dtype == torch.bfloat16 and W.grad.dtype == torch.bfloat16
+    # dH's split-K reduce-adds land in any order: compare up to bf16 rounding
+    ref = (3.0 * dH).to(torch.bfloat16).float()
+    assert rel_fro(h.grad.float().cpu().numpy(), ref.cpu().numpy()) < 1e-2 * 2 ** -6
+    assert torch.equal(W.grad, (3.0 * dW).to(torch.bfloat16))
+    o = oracle.oracle_from_inputs(inp)
+    assert rel_fro(h.grad.float().cpu().numpy(), 3.0 * o["dH"]) < GRAD_RTOL
+    assert rel_fro(W.grad.float().cpu().numpy(), 3.0 * o["dW"]) < GRAD_RTOL
