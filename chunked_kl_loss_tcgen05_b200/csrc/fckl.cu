@@ -553,14 +553,16 @@ fckl_status run(const Request& q) {
     if (!make_map(&mapD_k, dlog_c, L.V, cap, L.Vp * 2, BK, CM)) return FCKL_ERR_CUDA;
     if (!make_map(&mapdH, dH_c, L.H, cap, L.H * 4, 32, 32, true)) return FCKL_ERR_CUDA;
     const long long tiles_h = MT * NTh;
-    const int S = choose_split(tiles_h, KBv, pairs);
+    // A compacted chunk's row count is only known on the device: the kernel
+    // picks the split there (S = 0) and the launch covers every pair.
+    const int S = compact ? 0 : choose_split(tiles_h, KBv, pairs);
     SchedArgs sa_h{SCHED_SPLIT_K, (int)NTh, (int)KBv, S, 0, rc, 0, w3d, 0, narrow_h};
     EpiDH::Params ph{H, invT, ctl};
     {
       ProfScope ps(K_DH, st, gemm_flops,
                    2.0 * nr * (double)L.V + 2.0 * (double)L.V * L.H + 4.0 * nr * L.H);
       gemm_pair_kernel<EpiDH, false, true>
-          <<<grid_for(tiles_h * S), GEMM_THREADS, pair_smem_bytes<EpiDH>(), st>>>(
+          <<<S > 0 ? grid_for(tiles_h * S) : 2 * pairs, GEMM_THREADS, pair_smem_bytes<EpiDH>(), st>>>(
               mapD_k, mapW_mn, mapdH, ph, sa_h, ca);
     }
     if (list) {

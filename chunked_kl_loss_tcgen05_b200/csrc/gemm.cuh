@@ -30,6 +30,8 @@
 //   B MN-major : B[n, k] contiguous in n  -> two TMA boxes {64 n, 64 k}
 #pragma once
 
+#include <climits>
+
 #include "ptx.cuh"
 
 namespace fckl {
@@ -95,7 +97,7 @@ struct SchedArgs {
   int kind;
   int NT;      // vocab tiles (SCHED_VOCAB_MAJOR) / column tiles (SCHED_SPLIT_K, SCHED_TILES)
   int KB;      // k-blocks of the reduction (SCHED_VOCAB_MAJOR, SCHED_SPLIT_K)
-  int S;       // split-K factor (SCHED_SPLIT_K)
+  int S;       // split-K factor (SCHED_SPLIT_K); 0: chosen on the device from the row count
   int MT;      // row tiles of M (SCHED_TILES: M is the vocabulary)
   RowCount rc; // the launch's rows: M of the first two kinds, K of SCHED_TILES
   // MN-major operands: 1 = the map is 3-D {64, k, MN/64}, so that one box
@@ -111,6 +113,23 @@ __device__ __forceinline__ bool narrow_unit(const SchedArgs& a, const Work& w) {
   return a.narrow_tail && w.nt == a.NT - 1;
 }
 
+// Split-K factor for `tiles` output tiles of KB k-blocks on `slots` CTA pairs:
+// minimise waves * (k-blocks per unit + a fixed cost of 6 per unit).  Used on
+// the device when the row count (hence the tile count) is only known there;
+// the host applies the same model when it knows the rows.
+__device__ __forceinline__ int choose_split_dev(int tiles, int KB, int slots) {
+  if (tiles <= 0 || KB <= 0) return 1;
+  int best = 1;
+  long long best_cost = LLONG_MAX;
+  const int smax = KB < 128 ? KB : 128;
+  for (int S = 1; S <= smax; ++S) {
+    const long long waves = ((long long)tiles * S + slots - 1) / slots;
+    const long long cost = waves * ((KB + S - 1) / S + 6);
+    if (cost < best_cost) { best_cost = cost; best = S; }
+  }
+  return best;
+}
+
 // Cluster c of G takes units c, c+G, c+2G, ...  In every order above, the
 // clusters running at the same moment touch a narrow band of the streamed
 // operand, so it is read from DRAM about once and reused from L2.
@@ -118,8 +137,10 @@ struct PairSched {
   long long u, total;
   SchedArgs a;
   int G, rows, MT, tiles, KB;
-  __device__ void init(const SchedArgs& args, int cluster, int nclusters) {
+  // S_dev: the split factor the CTA chose on the device (used when a.S == 0).
+  __device__ void init(const SchedArgs& args, int cluster, int nclusters, int S_dev) {
     a = args; G = nclusters; u = cluster;
+    if (a.kind == SCHED_SPLIT_K && a.S == 0) a.S = S_dev;
     rows = a.rc.get();
     const int row_tiles = (rows + PM - 1) / PM;
     if (a.kind == SCHED_VOCAB_MAJOR) {
@@ -182,6 +203,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
   uint64_t* drain = tempty + 2;          // [1]       MMA drain at exit        (even CTA's used)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   uint32_t* abort_flag = tmem_slot + 1;
+  int* split_slot = reinterpret_cast<int*>(abort_flag + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -201,6 +223,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     }
     mbar_init(smem_u32(drain), 1);
     *abort_flag = 0u;
+    // Split-K factor chosen here when only the device knows the rows; every
+    // role (and both CTAs of the pair, from the same inputs) uses this value.
+    *split_slot = (sa.kind == SCHED_SPLIT_K && sa.S == 0)
+                      ? choose_split_dev(((sa.rc.get() + PM - 1) / PM) * sa.NT, sa.KB, nclusters)
+                      : sa.S;
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
@@ -221,7 +248,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       PairSched sch;
-      sch.init(sa, cluster, nclusters);
+      sch.init(sa, cluster, nclusters, *split_slot);
       Work w;
       int stage = 0;
       uint32_t phase = 0;
@@ -278,7 +305,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     // ------------------------------------------------------------ MMA issuer
     if (leader && lane == 0) {
       PairSched sch;
-      sch.init(sa, cluster, nclusters);
+      sch.init(sa, cluster, nclusters, *split_slot);
       Work w;
       int stage = 0;
       uint32_t phase = 0;
@@ -334,7 +361,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     const int quarter = warp & 3;  // TMEM lanes [32*quarter, +32) belong to this warp
     const int r = quarter * 32 + lane;
     PairSched sch;
-    sch.init(sa, cluster, nclusters);
+    sch.init(sa, cluster, nclusters, *split_slot);
     Work w;
     int acc = 0;
     uint32_t acc_phase = 0;

@@ -231,7 +231,8 @@ def test_teacher_row_without_finite_logit_is_reported():
 
 # ------------------------------------------------ sampled sparse targets (RS-KD)
 @pytest.mark.parametrize("shape", [(300, 128, 2000, 24, 1.0, 128), (517, 64, 777, 64, 2.0, 0),
-                                   (256, 256, 4096, 100, 1.0, 64)])
+                                   (256, 256, 4096, 100, 1.0, 64),
+                                   (1024, 3072, 128256, 100, 1.0, 0)])  # 8K Llama H, V, K
 def test_sampled_target_teacher_full(shape):
     """Teacher given as sampled class weights (repeats allowed): p = w / sum w."""
     N, H, V, K, T, chunk = shape
