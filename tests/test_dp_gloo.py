@@ -1,4 +1,4 @@
-"""Row-sharded data parallelism, host logic on CPU: two gloo ranks each pass
+"""Row-sharded data parallelism, host logic on CPU: two or three gloo ranks each pass
 their own row shard through fused_kl_fwd_bwd_dp (with the fp64 oracle as the
 per-rank compute), and the all-reduced loss and dW plus the concatenated dH
 shards must equal the unsharded result."""
@@ -55,9 +55,10 @@ def _worker(rank, world, port, case, out_q):
         dist.destroy_process_group()
 
 
+@pytest.mark.parametrize("world", [2, 3])
 @pytest.mark.parametrize("case", [dict(N=37, H=16, V=60, K=5, T=1.5, mask_frac=0.2, seed=3),
                                   dict(N=8, H=8, V=30, K=3, T=1.0, mask_frac=0.0, seed=4)])
-def test_two_rank_row_sharding_matches_unsharded(case):
+def test_row_sharding_matches_unsharded(case, world):
     import sys
     sys.path.insert(0, ROOT)
     import oracle
@@ -65,19 +66,19 @@ def test_two_rank_row_sharding_matches_unsharded(case):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, case, q)) for r in range(2)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, case, q)) for r in range(world)]
     for p in procs:
         p.start()
     res = {}
-    for _ in range(2):
+    for _ in range(world):
         rank, loss, dH, dW = q.get(timeout=120)
         res[rank] = (loss, dH, dW)
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
     full = oracle.oracle_from_inputs(synth.make_custom(**case))
-    for r in range(2):
+    for r in range(world):
         np.testing.assert_allclose(res[r][0], full["loss"], rtol=1e-12)
         np.testing.assert_allclose(res[r][2], full["dW"], rtol=1e-10, atol=1e-16)
-    np.testing.assert_allclose(np.concatenate([res[0][1], res[1][1]]), full["dH"], rtol=1e-10,
-                               atol=1e-16)
+    np.testing.assert_allclose(np.concatenate([res[r][1] for r in range(world)]), full["dH"],
+                               rtol=1e-10, atol=1e-16)
