@@ -82,3 +82,47 @@ def test_row_sharding_matches_unsharded(case, world):
         np.testing.assert_allclose(res[r][2], full["dW"], rtol=1e-10, atol=1e-16)
     np.testing.assert_allclose(np.concatenate([res[r][1] for r in range(world)]), full["dH"],
                                rtol=1e-10, atol=1e-16)
+
+
+def _worker_leaves(rank, world, port, out_q):
+    import sys
+    sys.path.insert(0, ROOT)
+    import datetime
+    import torch
+    import torch.distributed as dist
+    from chunked_kl_loss_tcgen05_b200.dp import fused_kl_fwd_bwd_dp
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=10))
+    if rank == 1:  # this rank leaves between steps, before its first collective
+        out_q.put((rank, "left"))
+        out_q.close()
+        out_q.join_thread()
+        os._exit(0)
+
+    def compute(*a, **kw):
+        raise AssertionError("never reached: the count all-reduce fails first")
+
+    h = torch.zeros(4, 8)
+    try:
+        fused_kl_fwd_bwd_dp(h, torch.zeros(16, 8), torch.zeros(4, 2, dtype=torch.int32),
+                            torch.zeros(4, 2), None, compute=compute)
+        out_q.put((rank, "no error"))
+    except Exception as e:  # the peer is gone: the collective must fail, not hang
+        out_q.put((rank, "error: " + type(e).__name__))
+
+
+def test_lost_rank_fails_the_collective_instead_of_hanging():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker_leaves, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = dict(q.get(timeout=120) for _ in range(2))
+    for p in procs:
+        p.join(timeout=60)
+    assert got[1] == "left"
+    assert got[0].startswith("error"), got[0]
