@@ -86,6 +86,9 @@ EDGE = [
     ("temperature_2", 256, 256, 4096, 16, 2.0, 0.25, 64),
     ("one_row", 1, 64, 512, 3, 1.0, 0.0, 0),
     ("many_chunks", 1000, 64, 513, 7, 1.0, 0.05, 37),
+    ("k_equals_v", 64, 64, 200, 200, 1.0, 0.0, 0),       # the teacher covers the vocabulary
+    ("temperature_small", 256, 128, 3000, 16, 0.25, 0.1, 0),
+    ("temperature_large", 256, 128, 3000, 16, 8.0, 0.1, 0),
 ]
 
 
@@ -227,6 +230,34 @@ def test_teacher_row_without_finite_logit_is_reported():
     lg = inp.topk_logit.copy()
     lg[3, 2] = np.nan
     assert _raw_call(inp, logits=lg) == FCKL_ERR_BAD_TEACHER
+
+
+def test_partly_minus_inf_teacher_logits():
+    """-inf teacher logits are entries of probability 0 (a padded cache); rows
+    keep at least one finite logit."""
+    inp = synth.make_custom(300, 128, 2000, 16, T=1.0, sigma=2.0, mask_frac=0.1, seed=93,
+                            chunk=128)
+    rng = np.random.default_rng(93)
+    pad = rng.random(inp.topk_logit.shape) < 0.3
+    pad[:, 0] = False
+    inp.topk_logit[pad] = -np.inf
+    o = oracle.oracle_from_inputs(inp)
+    check_full(inp, run_gpu(inp), o)
+
+
+def test_masked_rows_with_invalid_teacher_data_are_ignored():
+    """A masked row takes no part in the loss: its ids and logits are not even
+    checked (the same call with clean masked rows gives the same result)."""
+    inp = synth.make_custom(200, 64, 700, 8, mask_frac=0.3, seed=94, chunk=64)
+    ref = run_gpu(inp)
+    m = inp.row_mask == 0
+    inp.topk_idx[m] = 700 + 5
+    inp.topk_idx[np.nonzero(m)[0][:3]] = -3
+    inp.topk_logit[m] = np.nan
+    assert _raw_call(inp) == FCKL_OK
+    g = run_gpu(inp)
+    assert g["loss"] == ref["loss"]
+    assert torch.equal(g["dW"], ref["dW"])
 
 
 # ------------------------------------------------ sampled sparse targets (RS-KD)
