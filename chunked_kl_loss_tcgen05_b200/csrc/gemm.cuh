@@ -25,9 +25,13 @@
 //
 // Operand majors (bf16, row-major global tensors), per CTA and stage:
 //   A K-major  : A[m, k] contiguous in k  -> TMA box {64 k, 128 m}
-//   A MN-major : A[m, k] contiguous in m  -> two TMA boxes {64 m, 64 k}
+//   A MN-major : A[m, k] contiguous in m  -> one 3-D box {64 m, 64 k, 2 chunks}
+//                (or two 2-D boxes {64 m, 64 k} when m's extent is not a
+//                multiple of 64)
 //   B K-major  : B[n, k] contiguous in k  -> TMA box {64 k, 128 n}
-//   B MN-major : B[n, k] contiguous in n  -> two TMA boxes {64 n, 64 k}
+//   B MN-major : B[n, k] contiguous in n  -> as A MN-major
+// A last column tile of at most 128 columns may run as N = 128 MMAs (each CTA
+// stages 64 columns of B); see SchedArgs::narrow_tail.
 #pragma once
 
 #include <climits>
