@@ -3,14 +3,21 @@
 
 One step = one fckl_fwd_bwd call over the whole workload (every chunk: teacher
 prep, fused projection + log-sum-exp, recompute + dlogits, dH and dW GEMMs).
-Default workload: the Llama-3.1-8B -> ~3B student shape at 8K context
-(N=8192, H=3072, V=128256, K=100, T=1, 5% rows masked).  Other configs are
-available with --config.
+Default workload: the largest single-GPU one, 256K tokens (N=262144, H=4096,
+V=128256, K=100, T=2, 10% rows masked, chunk 2048; "Knowledge Distillation 비용
+줄이기", section "chunked KL loss가 하는 일").  Other workloads: --config
+(0 tiny, 1 the 8K Llama-3.1-8B -> ~3B student shape, 2 the 32K toy output
+projection, 3 the gpt-oss-20b student shape); --rows shrinks a workload's row
+count (small cases for profiler captures).
 
-Under torchrun with N ranks every rank runs its own replica of the workload on
-its own GPU (no data-path collective; "scaling": "weak"); the timing is the max
-over ranks.  `--impl reference` times the fp64 CPU oracle instead, on a bounded
-sample of rows of the same workload, on rank 0 only.
+Under torchrun with N ranks (--mode dp, the default there) the ranks run
+row-sharded data parallelism: every rank holds one shard of N_rows rows of a
+global batch of N * N_rows rows ("scaling": "weak"), the ranks all-reduce the
+valid-row count, and the dW all-reduce overlaps the last dW GEMM
+(chunked_kl_loss_tcgen05_b200.dp).  --mode replicas runs independent replicas
+with no data-path collective.  Timing is the max over ranks.
+`--impl reference` times the fp64 CPU oracle instead, on a bounded sample of
+rows of the same workload, on rank 0 only.
 """
 from __future__ import annotations
 
@@ -22,6 +29,8 @@ import subprocess
 import sys
 import tempfile
 import time
+
+import dataclasses
 
 import numpy as np
 
@@ -37,11 +46,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum, mean over the
 # launches of one call) from the ncu capture of the current kernels on this workload,
 # summarised under profiles/.  Reset an entry to None when its kernel changes.
-MEASURED_TRAFFIC = {
-    "llama8b_to_3b_8k_N8192_H3072_V128256_K100": {
-        "fwd_logits_lse": 1.001e9, "bwd_dlogits": 2.326e9, "dH_gemm": 7.038e9,
-        "dW_gemm": 4.063e9},
-}
+MEASURED_TRAFFIC = {}
 
 
 def load_peaks():
@@ -58,9 +63,20 @@ def load_peaks():
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--config", type=int, default=4)
+    ap.add_argument("--rows", type=int, default=0,
+                    help="use only this many rows of the workload (0 = all; same H, V, K, T, "
+                         "chunk and mask fraction)")
+    ap.add_argument("--dw-rows", type=int, default=0,
+                    help="group chunks so that each dW GEMM covers at least this many rows "
+                         "(fckl_problem.dw_rows; 0 = one dW GEMM per chunk)")
+    ap.add_argument("--mode", default="", choices=["", "dp", "replicas"],
+                    help="multi-GPU mode under torchrun (default dp)")
+    ap.add_argument("--dp-slices", type=int, default=8,
+                    help="dp mode: vocabulary slices of the last dW GEMM whose all-reduce "
+                         "overlaps the rest")
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--graph", action="store_true",
@@ -70,6 +86,8 @@ def parse():
     ap.add_argument("--profile-json", default="")
     ap.add_argument("--mem-sweep", action="store_true",
                     help="print peak device memory vs sequence length instead of timing")
+    ap.add_argument("--sweep-chunk", type=int, default=2048,
+                    help="--mem-sweep: rows per chunk")
     ap.add_argument("--vs-cublas", type=float, default=0.0, metavar="SECONDS",
                     help="instead of the contract line: run the fused step and the four plain "
                          "cuBLAS GEMMs of the same shapes back to back for SECONDS each, clocks "
@@ -82,17 +100,34 @@ def dist_env():
             int(os.environ.get("WORLD_SIZE", "1")))
 
 
-def workload_config(cfg: synth.Config, C: int) -> dict:
+def workload(args) -> synth.Config:
+    """The selected workload, optionally cut to its first --rows rows."""
+    cfg = synth.CONFIGS[args.config]
+    if args.rows and args.rows != cfg.N:
+        cfg = dataclasses.replace(cfg, N=int(args.rows), name=f"{cfg.name}_rows{int(args.rows)}")
+    return cfg
+
+
+def workload_config(cfg: synth.Config, C: int, dw_rows: int = 0) -> dict:
     return {"workload": cfg.name, "N_rows": cfg.N, "H": cfg.H, "V": cfg.V, "K": cfg.K, "T": cfg.T,
-            "chunk": C, "mask_frac": cfg.mask_frac,
+            "chunk": C, "dw_rows": dw_rows, "mask_frac": cfg.mask_frac,
             "l2": "inputs larger than L2 (W alone is %.0f MB > 126 MB)" % (cfg.V * cfg.H * 2 / 1e6),
             "data": "synthetic seeded (synth recipe)"}
 
 
-def resolved_chunk(cfg: synth.Config) -> int:
-    """The chunk the library uses for this workload (host arithmetic only)."""
-    from chunked_kl_loss_tcgen05_b200 import FcklProblem, fckl_resolved_chunk
-    return fckl_resolved_chunk(FcklProblem(cfg.N, cfg.H, cfg.V, cfg.K, cfg.T, cfg.chunk))
+def library_chunk(cfg: synth.Config) -> int:
+    """The chunk the library resolves for this workload, restated here so that
+    the oracle arm never loads the library: an explicit chunk capped at N, or
+    (chunk = 0) the largest multiple of 128 rows whose bf16 dlogits block
+    [chunk, V rounded up to 64] fits in 1 GiB, at least 128, capped at N rounded
+    up to 64, then at N (tests/test_boundary.py checks that both agree)."""
+    C = cfg.chunk
+    if C == 0:
+        Vp = (cfg.V + 63) // 64 * 64
+        C = (1 << 30) // (Vp * 2) // 128 * 128
+        C = max(C, 128)
+        C = min(C, (cfg.N + 63) // 64 * 64)
+    return min(C, cfg.N)
 
 
 # ------------------------------------------------------------------ oracle arm
@@ -114,7 +149,9 @@ def cpu_cores():
 
 
 def auto_cpu_rows(cfg):
-    # ~6*H*V fp64 flops per row; aim at ~10 s of host work at ~100 GFLOP/s
+    """Rows of the oracle sample: ~6*H*V fp64 flops per row (logits, dH, dW
+    contribution), ~1 TFLOP per sample (a few seconds on a many-core host).
+    The CUDA arm's cpu_baseline and the reference arm use the same sample."""
     per_row = 6.0 * cfg.H * cfg.V
     return int(max(16, min(1024, 1e12 / per_row)))
 
@@ -123,9 +160,9 @@ def run_reference(args):
     rank, _, world = dist_env()
     if rank != 0:
         return 0
-    cfg = synth.CONFIGS[args.config]
+    cfg = workload(args)
     inp = synth.make_inputs(cfg)
-    n_rows = args.cpu_rows or max(8, auto_cpu_rows(cfg) // 8)
+    n_rows = args.cpu_rows or auto_cpu_rows(cfg)
     times = []
     for i in range(args.warmup + args.steps):
         rps, n, dt = oracle_rows_per_sec(inp, n_rows)
@@ -138,8 +175,9 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": dict(workload_config(cfg, resolved_chunk(cfg)),
-                           parallelism=f"replicas{world}", flush="inputs larger than L2"),
+            "config": dict(workload_config(cfg, library_chunk(cfg), args.dw_rows),
+                           parallelism=f"oracle on rank 0 of {world}",
+                           flush="inputs larger than L2"),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_cores(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -199,7 +237,7 @@ class ClockSampler:
 def run_cuda(args):
     import torch
     import torch.distributed as dist
-    from chunked_kl_loss_tcgen05_b200 import (FcklProblem, fckl_resolved_chunk,
+    from chunked_kl_loss_tcgen05_b200 import (FcklProblem, fckl_check, fckl_resolved_chunk,
                                               fckl_profile_begin, fckl_profile_end)
     from chunked_kl_loss_tcgen05_b200.torch_api import (alloc_workspace, arrays_to_device,
                                                         fused_kl_fwd_bwd)
@@ -207,6 +245,7 @@ def run_cuda(args):
     rank, local, world = dist_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    mode = "single" if world == 1 else (args.mode or "dp")
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
@@ -216,9 +255,11 @@ def run_cuda(args):
         if world > 1:
             dist.barrier()
 
-    cfg = synth.CONFIGS[args.config]
+    cfg = workload(args)
+    # Every rank's shard (dp) or replica is the same seeded workload: the work
+    # and its cost do not depend on the values.
     inp = synth.make_inputs(cfg)
-    prob = FcklProblem(cfg.N, cfg.H, cfg.V, cfg.K, cfg.T, cfg.chunk)
+    prob = FcklProblem(cfg.N, cfg.H, cfg.V, cfg.K, cfg.T, cfg.chunk, dw_rows=args.dw_rows)
     C = fckl_resolved_chunk(prob)
     n_valid = int(inp.row_mask.sum())
     d = arrays_to_device(inp.hidden, inp.W, inp.topk_idx, inp.topk_logit, inp.row_mask, dev)
@@ -229,10 +270,17 @@ def run_cuda(args):
     outs = (torch.empty(1, device=dev), torch.empty(cfg.N, cfg.H, device=dev),
             torch.empty(cfg.V, cfg.H, device=dev))
 
-    def step():
-        return fused_kl_fwd_bwd(*d, T=cfg.T, chunk=cfg.chunk, workspace=ws, check=False, out=outs)
+    if mode == "dp":
+        from chunked_kl_loss_tcgen05_b200.dp import fused_kl_fwd_bwd_dp
 
-    from chunked_kl_loss_tcgen05_b200 import fckl_check
+        def step():
+            return fused_kl_fwd_bwd_dp(*d, T=cfg.T, chunk=cfg.chunk, workspace=ws,
+                                       n_slices=args.dp_slices, out=outs, dw_rows=args.dw_rows)
+    else:
+        def step():
+            return fused_kl_fwd_bwd(*d, T=cfg.T, chunk=cfg.chunk, workspace=ws, check=False,
+                                    out=outs, dw_rows=args.dw_rows)
+
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -274,10 +322,7 @@ def run_cuda(args):
     if st != 0:
         raise SystemExit(f"device error in the timed steps: status {st}")
 
-    t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_total = float(t.item())
+    ms_total = max_over_ranks(torch, dev, ms_total, world)
     ms_step = ms_total / args.steps
     tokens = cfg.N * world
     value = tokens / (ms_step / 1e3)
@@ -285,41 +330,48 @@ def run_cuda(args):
     tflops = flops_step * world / (ms_step / 1e3) / 1e12
 
     peaks = load_peaks()
+    burst = peaks["bf16_tflops"]
+    sustained = peaks.get("bf16_tflops_sustained") or burst
     # dominant kernel: its launches were event-timed inside the timed region
     bd_total = sum(p["total_ms"] for p in breakdown) or 1.0
     dom = max(prof, key=lambda p: p["total_ms"]) if prof else None
-    prof_total = bd_total
     roofline = None
     if dom is not None:
         avg_ms = dom["total_ms"] / dom["launches"]
+        share = dom["total_ms"] / args.steps / ms_step
+        traffic = MEASURED_TRAFFIC.get(cfg.name, {}).get(dom["name"])
         if dom["flops"] > 0:
-            peak = peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"]
             ach = dom["flops"] / dom["launches"] / (avg_ms / 1e3) / 1e12
-            roofline = {"kernel": dom["name"], "bound": "tensor", "achieved": ach, "peak": peak,
-                        "unit": "TFLOP/s", "frac": ach / peak,
-                        "peak_kind": f"bf16_tflops_sustained ({peaks['source']})",
-                        "traffic": MEASURED_TRAFFIC.get(cfg.name, {}).get(dom["name"]),
+            roofline = {"kernel": dom["name"], "bound": "tensor", "achieved": ach, "peak": burst,
+                        "unit": "TFLOP/s", "frac": ach / burst,
+                        "peak_kind": f"bf16_tflops burst ({peaks['source']})",
+                        "frac_of_sustained_peak": ach / sustained,
+                        "sustained_peak": sustained,
+                        "traffic": traffic,
                         "algorithmic_bytes": dom["bytes"] / dom["launches"],
-                        "share": dom["total_ms"] / args.steps / ms_step}
+                        "algorithmic_flops": dom["flops"] / dom["launches"],
+                        "launch_ms": avg_ms, "share": share}
         else:
             peak = peaks["hbm_gbs"]
             ach = dom["bytes"] / dom["launches"] / (avg_ms / 1e3) / 1e9
             roofline = {"kernel": dom["name"], "bound": "hbm", "achieved": ach, "peak": peak,
                         "unit": "GB/s", "frac": ach / peak, "peak_kind": f"hbm_gbs ({peaks['source']})",
-                        "traffic": MEASURED_TRAFFIC.get(cfg.name, {}).get(dom["name"]),
-                        "share": dom["total_ms"] / args.steps / ms_step}
-    kernels = [{"name": p["name"], "launches": p["launches"], "ms_per_step": p["total_ms"] / 2,
+                        "traffic": traffic, "launch_ms": avg_ms, "share": share}
+    kernels = [{"name": p["name"], "launches": p["launches"] // 2, "ms_per_step": p["total_ms"] / 2,
                 "share": p["total_ms"] / bd_total,
                 "tflops": (p["flops"] / (p["total_ms"] / 1e3) / 1e12) if p["flops"] else None}
                for p in breakdown]
 
     graph = None
-    if args.graph:
+    if args.graph and mode != "dp":
         graph = measure_graph(torch, dev, step, args.steps, cfg, world)
 
     e2e = None
     if not args.no_e2e:
-        e2e = measure_e2e(torch, dev, inp, cfg, ws, args.steps, world, outs)
+        if mode == "dp":
+            e2e = measure_e2e_dp(torch, dev, inp, cfg, ws, args, world, outs, d)
+        else:
+            e2e = measure_e2e(torch, dev, inp, cfg, ws, args.steps, world, outs, args.dw_rows)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -330,17 +382,19 @@ def run_cuda(args):
                          f"{dt:.1f} s"}
 
     if rank == 0:
+        par = {"single": "1 GPU", "replicas": f"replicas{world}",
+               "dp": f"dp{world} (row shards, dW all-reduce overlapped)"}[mode]
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16", "data": "synthetic",
-                "config": dict(workload_config(cfg, C), parallelism=f"replicas{world}",
-                               flush="inputs larger than L2"),
+                "config": dict(workload_config(cfg, C, args.dw_rows), parallelism=par,
+                               global_batch=cfg.N * world, flush="inputs larger than L2"),
                 "tflops": tflops,
-                "frac_of_peak": {"measured_burst": tflops / world / peaks["bf16_tflops"],
-                                 "measured_sustained": tflops / world / peaks.get(
-                                     "bf16_tflops_sustained", peaks["bf16_tflops"]),
+                "frac_of_peak": {"measured_burst": tflops / world / burst,
+                                 "measured_sustained": tflops / world / sustained,
                                  "dense_spec_2250": tflops / world / 2250.0},
+                "peaks_source": peaks["source"],
                 "peak_mem_gib": peak_gib, "loss": loss_val,
                 "roofline": roofline, "kernels": kernels,
                 "cpu_baseline": cpu, "e2e": e2e, "clocks": clk, "graph": graph,
@@ -391,7 +445,7 @@ def measure_graph(torch, dev, step, steps, cfg, world):
     return {"value": cfg.N * world / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms}
 
 
-def measure_e2e(torch, dev, inp, cfg, ws, steps, world, outs):
+def measure_e2e(torch, dev, inp, cfg, ws, steps, world, outs, dw_rows=0):
     """Same metric through the host-input C-ABI call: every step the library
     copies that step's inputs (hidden states, teacher top-K ids and logits, row
     mask) from pinned host memory to the device, overlapped chunk by chunk with
@@ -405,7 +459,7 @@ def measure_e2e(torch, dev, inp, cfg, ws, steps, world, outs):
             "row_mask": torch.from_numpy(inp.row_mask).pin_memory()}
     W = torch.from_numpy(inp.W.view(np.int16)).view(torch.bfloat16).to(dev)
     h2d = sum(v.numel() * v.element_size() for v in host.values())
-    prob = FcklProblem(cfg.N, cfg.H, cfg.V, cfg.K, cfg.T, cfg.chunk)
+    prob = FcklProblem(cfg.N, cfg.H, cfg.V, cfg.K, cfg.T, cfg.chunk, dw_rows=dw_rows)
     hws = alloc_host_workspace(prob, dev)
     loss_host = torch.empty(1, dtype=torch.float32, pin_memory=True)
     out = (outs[1], outs[2])
@@ -413,7 +467,7 @@ def measure_e2e(torch, dev, inp, cfg, ws, steps, world, outs):
     def call():
         return fused_kl_fwd_bwd_host(host["hidden"], W, host["topk_idx"], host["topk_logit"],
                                      host["row_mask"], T=cfg.T, chunk=cfg.chunk, workspace=hws,
-                                     out=out, loss_host=loss_host, check=False)
+                                     out=out, loss_host=loss_host, check=False, dw_rows=dw_rows)
     for _ in range(2):
         call()
     torch.cuda.synchronize()
@@ -431,14 +485,55 @@ def measure_e2e(torch, dev, inp, cfg, ws, steps, world, outs):
             "path": "fckl_fwd_bwd_host (inputs pinned on the host, W resident)"}
 
 
+def measure_e2e_dp(torch, dev, inp, cfg, ws, args, world, outs, d):
+    """dp mode end to end through the data-parallel API: every step copies the
+    rank's shard (hidden states, teacher top-K ids and logits, row mask) from
+    pinned host memory into the device buffers, runs fused_kl_fwd_bwd_dp
+    (valid-count and dW all-reduces included) and reads the loss back."""
+    from chunked_kl_loss_tcgen05_b200.dp import fused_kl_fwd_bwd_dp
+    host = [torch.from_numpy(inp.hidden.view(np.int16)).view(torch.bfloat16).pin_memory(), None,
+            torch.from_numpy(inp.topk_idx).pin_memory(),
+            torch.from_numpy(inp.topk_logit).pin_memory(),
+            torch.from_numpy(inp.row_mask).pin_memory()]
+    h2d = sum(t.numel() * t.element_size() for t in host if t is not None)
+    loss_host = torch.empty(1, dtype=torch.float32, pin_memory=True)
+
+    def call():
+        for i, t in enumerate(host):
+            if t is not None:
+                d[i].copy_(t, non_blocking=True)
+        loss, _, _ = fused_kl_fwd_bwd_dp(*d, T=cfg.T, chunk=cfg.chunk, workspace=ws,
+                                         n_slices=args.dp_slices, out=outs, dw_rows=args.dw_rows)
+        loss_host.copy_(loss, non_blocking=True)
+        torch.cuda.current_stream(dev).synchronize()
+        return float(loss_host[0])
+    for _ in range(2):
+        call()
+    torch.cuda.synchronize()
+    import torch.distributed as dist
+    dist.barrier()
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(torch, dev, e0.elapsed_time(e1) / args.steps, world)
+    return {"value": cfg.N * world / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": 4, "steps": args.steps,
+            "path": "fused_kl_fwd_bwd_dp after host->device copies of the shard from pinned memory"}
+
+
 def run_mem_sweep(args):
     """Peak device memory of one fused forward+backward call vs sequence length
-    at the 32K toy-projection shape (H=4096, V=128256, K=100, chunk=2048):
-    inputs, outputs and workspace all counted (torch.cuda.max_memory_allocated)."""
+    at the 32K toy-projection shape (H=4096, V=128256, K=100, chunk
+    --sweep-chunk): inputs, outputs and workspace all counted
+    (torch.cuda.max_memory_allocated)."""
     import torch
     from chunked_kl_loss_tcgen05_b200.torch_api import fused_kl_fwd_bwd
     torch.cuda.set_device(0)
-    H, V, K, C = 4096, 128256, 100, 2048
+    H, V, K, C = 4096, 128256, 100, args.sweep_chunk
     pts = []
     for S in (8192, 16384, 32768, 65536, 131072, 262144):
         torch.cuda.empty_cache()
@@ -450,7 +545,8 @@ def run_mem_sweep(args):
         lg = torch.randn(S, K, device="cuda", generator=g) * 3
         torch.cuda.synchronize()
         torch.cuda.reset_peak_memory_stats()  # inputs stay counted, their fp32 temporaries do not
-        loss, _, dH, dW = fused_kl_fwd_bwd(hidden, W, ids, lg, None, T=1.0, chunk=C)
+        loss, _, dH, dW = fused_kl_fwd_bwd(hidden, W, ids, lg, None, T=1.0, chunk=C,
+                                           dw_rows=args.dw_rows)
         torch.cuda.synchronize()
         peak = (torch.cuda.max_memory_allocated() - base) / 2**30
         pts.append((S, peak))
@@ -459,7 +555,8 @@ def run_mem_sweep(args):
     ys = np.array([p[1] for p in pts], dtype=np.float64)
     b, a = np.polyfit(xs, ys, 1)
     r2 = 1 - ((ys - (a + b * xs)) ** 2).sum() / ((ys - ys.mean()) ** 2).sum()
-    line = {"metric": "peak GiB vs seq len (fused fwd+bwd, H=4096 V=128256 K=100 chunk=2048)",
+    line = {"metric": f"peak GiB vs seq len (fused fwd+bwd, H=4096 V=128256 K=100 chunk={C}, "
+                      f"dw_rows={args.dw_rows})",
             "points": [{"S": s, "peak_gib": round(p, 4)} for s, p in pts],
             "fit": {"intercept_gib": a, "slope_kib_per_row": b * 2**20, "r2": r2}}
     print(json.dumps(line), flush=True)
@@ -477,10 +574,10 @@ def run_vs_cublas(args):
     from chunked_kl_loss_tcgen05_b200.torch_api import (alloc_workspace, arrays_to_device,
                                                         fused_kl_fwd_bwd)
     torch.cuda.set_device(0)
-    cfg = synth.CONFIGS[args.config]
+    cfg = workload(args)
     inp = synth.make_inputs(cfg)
     d = arrays_to_device(inp.hidden, inp.W, inp.topk_idx, inp.topk_logit, inp.row_mask)
-    prob = FcklProblem(cfg.N, cfg.H, cfg.V, cfg.K, cfg.T, cfg.chunk)
+    prob = FcklProblem(cfg.N, cfg.H, cfg.V, cfg.K, cfg.T, cfg.chunk, dw_rows=args.dw_rows)
     C = fckl_resolved_chunk(prob)
     ws = alloc_workspace(prob, d[0].device)
     outs = (torch.empty(1, device="cuda"), torch.empty(cfg.N, cfg.H, device="cuda"),
@@ -488,7 +585,8 @@ def run_vs_cublas(args):
     n_valid = int(inp.row_mask.sum())
 
     def fused():
-        fused_kl_fwd_bwd(*d, T=cfg.T, chunk=cfg.chunk, workspace=ws, check=False, out=outs)
+        fused_kl_fwd_bwd(*d, T=cfg.T, chunk=cfg.chunk, workspace=ws, check=False, out=outs,
+                         dw_rows=args.dw_rows)
 
     h = d[0][:C].contiguous()
     W = d[1]

@@ -52,11 +52,13 @@ class FcklProblem(ctypes.Structure):
     """Mirror of ``fckl_problem``."""
     _fields_ = [("N", ctypes.c_int64), ("H", ctypes.c_int64), ("V", ctypes.c_int64),
                 ("K", ctypes.c_int32), ("T", ctypes.c_float), ("chunk", ctypes.c_int64),
-                ("teacher", ctypes.c_int32), ("n_valid_total", ctypes.c_int64)]
+                ("teacher", ctypes.c_int32), ("n_valid_total", ctypes.c_int64),
+                ("dw_rows", ctypes.c_int64)]
 
-    def __init__(self, N, H, V, K, T=1.0, chunk=0, teacher=FCKL_TEACHER_LOGITS, n_valid_total=0):
+    def __init__(self, N, H, V, K, T=1.0, chunk=0, teacher=FCKL_TEACHER_LOGITS, n_valid_total=0,
+                 dw_rows=0):
         super().__init__(int(N), int(H), int(V), int(K), float(T), int(chunk), int(teacher),
-                         int(n_valid_total))
+                         int(n_valid_total), int(dw_rows))
 
 
 class FcklKernelStat(ctypes.Structure):

@@ -24,8 +24,6 @@ namespace {
 constexpr size_t kAlign = 256;
 constexpr int kMaxDevices = 64;
 
-constexpr long long kDwRows = 4096;  // minimum reduction depth of a dW launch (rows)
-
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
 
@@ -44,6 +42,7 @@ bool valid_problem(const fckl_problem* p) {
   if (p->N > INT32_MAX || p->H > INT32_MAX || p->V > INT32_MAX) return false;
   if (p->teacher != FCKL_TEACHER_LOGITS && p->teacher != FCKL_TEACHER_PROBS) return false;
   if (p->n_valid_total < 0 || p->n_valid_total > INT32_MAX) return false;
+  if (p->dw_rows < 0 || p->dw_rows > INT32_MAX) return false;
   return true;
 }
 
@@ -55,9 +54,9 @@ long long resolve_chunk(const fckl_problem* p) {
   const long long Vp = align_up((size_t)p->V, 64);
   long long C = p->chunk;
   if (C == 0) {
-    // 1 GiB: the dW GEMM reduces over >= 4096 rows of dlogits anyway, so at
-    // V = 128K a 4096-row chunk costs no more workspace than smaller chunks
-    // grouped for dW, and halves the launches (and their tail waves).
+    // 1 GiB of bf16 dlogits: at V = 128K a 4096-row chunk, deep enough that
+    // one dW read-modify-write (V*H*8 bytes) per chunk stays well under the
+    // chunk's dW tensor-core time, with few launches (and tail waves).
     const long long budget = 1024ll << 20;
     C = budget / (Vp * 2) / 128 * 128;
     C = std::max(C, 128ll);
@@ -77,9 +76,12 @@ Layout make_layout(const fckl_problem* p, bool full = true) {
   L.C = resolve_chunk(p);
   L.nchunks = cdiv(L.N, L.C);
   // The dW GEMM reduces over the rows of its dlogits block, and each launch
-  // reads and writes dW once (fp32, V*H*8 bytes).  Small chunks are grouped
-  // so that one dW launch covers at least kDwRows rows.
-  L.G = std::min<long long>(L.nchunks, std::max<long long>(1, cdiv(kDwRows, L.C)));
+  // reads and writes dW once (fp32, V*H*8 bytes).  By default every chunk
+  // runs its own dW GEMM, so the workspace holds one chunk of dlogits; a
+  // caller may group chunks (dw_rows) so that one dW launch covers at least
+  // dw_rows rows, at the cost of keeping the group's dlogits live together.
+  L.G = std::min<long long>(L.nchunks,
+                            std::max<long long>(1, cdiv((long long)p->dw_rows, L.C)));
   L.NT = cdiv(L.V, BN);
   size_t off = align_up(sizeof(DeviceCtl), kAlign);
   auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes, kAlign); return o; };
@@ -729,11 +731,14 @@ fckl_status fckl_fwd_noalloc(const fckl_problem* prob, const void* hidden, const
   if (device_status && !aligned(device_status, 4)) return FCKL_ERR_INVALID_ARG;
   fckl_problem q = *prob;
   long long C = resolve_chunk(prob);
-  for (;;) {  // the largest chunk (or the caller's chunk) whose scratch fits
+  // The caller's chunk, or the automatic one; if its scratch does not fit
+  // (automatic chunk only), the largest multiple of PM rows below it that fits.
+  for (;;) {
     q.chunk = C;
     if (make_layout(&q, false).total <= kStaticScratchBytes) break;
-    if (prob->chunk != 0 || C <= PM) return FCKL_ERR_WORKSPACE;
-    C = std::max<long long>(PM, C / 2 / PM * PM);
+    if (prob->chunk != 0) return FCKL_ERR_WORKSPACE;
+    C = (C - 1) / PM * PM;
+    if (C < PM) return FCKL_ERR_WORKSPACE;
   }
   void* scratch = static_scratch();
   if (scratch == nullptr) return FCKL_ERR_CUDA;

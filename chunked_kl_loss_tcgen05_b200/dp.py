@@ -22,7 +22,8 @@ def shard_rows(N: int, rank: int, world: int) -> tuple:
 
 
 def fused_kl_fwd_bwd_dp(hidden, W, topk_idx, topk_logit, row_mask=None, T=1.0, chunk=0,
-                        teacher=0, group=None, compute=None, workspace=None, n_slices=4):
+                        teacher=0, group=None, compute=None, workspace=None, n_slices=4,
+                        out=None, dw_rows=0):
     """Full-batch loss and dW (identical on every rank) and the dH rows of this
     rank's shard.
 
@@ -32,13 +33,14 @@ def fused_kl_fwd_bwd_dp(hidden, W, topk_idx, topk_logit, row_mask=None, T=1.0, c
     the last slice's all-reduce follows the GEMM.  ``compute`` replaces the
     fused call (host-logic tests): it receives ``n_valid_total`` (the global
     N_v) and returns (loss[1], dH, dW, slices) with slices a list of (row0,
-    row1, event or None) covering dW's rows in order."""
+    row1, event or None) covering dW's rows in order.  ``out`` (loss, dH, dW)
+    and ``dw_rows`` are passed to the fused call."""
     if compute is None:
         from .torch_api import fused_kl_fwd_bwd_sliced
 
         def compute(h, w, i, l, m, **kw):
             return fused_kl_fwd_bwd_sliced(h, w, i, l, m, workspace=workspace,
-                                           n_slices=n_slices, **kw)
+                                           n_slices=n_slices, out=out, dw_rows=dw_rows, **kw)
     dev = hidden.device
     local = (row_mask != 0).sum() if row_mask is not None else torch.tensor(hidden.shape[0])
     count = local.to(device=dev, dtype=torch.int64).reshape(1)

@@ -29,11 +29,12 @@ def _bits(t: torch.Tensor) -> torch.Tensor:
     raise TypeError(f"expected bfloat16 (or its uint16 bits), got {t.dtype}")
 
 
-def make_problem(hidden, W, topk_idx, T=1.0, chunk=0, teacher=0, n_valid_total=0) -> FcklProblem:
+def make_problem(hidden, W, topk_idx, T=1.0, chunk=0, teacher=0, n_valid_total=0,
+                 dw_rows=0) -> FcklProblem:
     N, H = hidden.shape
     V = W.shape[0]
     K = topk_idx.shape[1]
-    return FcklProblem(N, H, V, K, T, chunk, teacher, n_valid_total)
+    return FcklProblem(N, H, V, K, T, chunk, teacher, n_valid_total, dw_rows)
 
 
 def alloc_workspace(prob: FcklProblem, device) -> torch.Tensor:
@@ -56,15 +57,17 @@ def _check_inputs(hidden, W, topk_idx, topk_logit, row_mask):
 
 def fused_kl_fwd_bwd(hidden, W, topk_idx, topk_logit, row_mask=None, T=1.0, chunk=0,
                      workspace=None, want_row_loss=False, check=True, out=None, teacher=0,
-                     n_valid_total=0):
+                     n_valid_total=0, dw_rows=0):
     """Returns (loss[1], row_loss[N] or None, dH[N,H] fp32, dW[V,H] fp32).
 
     ``out``: optional (loss, dH, dW) tensors to write into instead of allocating.
     ``n_valid_total``: N_v for the mean and gradient scale when these rows are one
-    shard of a larger batch (0 = the valid rows of this call)."""
+    shard of a larger batch (0 = the valid rows of this call).
+    ``dw_rows``: group chunks so that each dW GEMM covers at least this many
+    rows (0 = one dW GEMM per chunk)."""
     hidden, W = _bits(hidden), _bits(W)
     _check_inputs(hidden, W, topk_idx, topk_logit, row_mask)
-    prob = make_problem(hidden, W, topk_idx, T, chunk, teacher, n_valid_total)
+    prob = make_problem(hidden, W, topk_idx, T, chunk, teacher, n_valid_total, dw_rows)
     dev = hidden.device
     if workspace is None:
         workspace = alloc_workspace(prob, dev)
@@ -95,14 +98,15 @@ def fused_kl_fwd_bwd(hidden, W, topk_idx, topk_logit, row_mask=None, T=1.0, chun
 
 
 def fused_kl_fwd_bwd_sliced(hidden, W, topk_idx, topk_logit, row_mask=None, T=1.0, chunk=0,
-                            workspace=None, n_slices=4, teacher=0, n_valid_total=0, out=None):
+                            workspace=None, n_slices=4, teacher=0, n_valid_total=0, out=None,
+                            dw_rows=0):
     """fused_kl_fwd_bwd whose last dW launch is split into ``n_slices``
     vocabulary slices.  Returns (loss[1], dH, dW, slices) with slices a list of
     (row0, row1, event): dW[row0:row1] is final once ``event`` (a
     torch.cuda.Event recorded on the current stream) has completed."""
     hidden, W = _bits(hidden), _bits(W)
     _check_inputs(hidden, W, topk_idx, topk_logit, row_mask)
-    prob = make_problem(hidden, W, topk_idx, T, chunk, teacher, n_valid_total)
+    prob = make_problem(hidden, W, topk_idx, T, chunk, teacher, n_valid_total, dw_rows)
     dev = hidden.device
     if workspace is None:
         workspace = alloc_workspace(prob, dev)
@@ -160,7 +164,7 @@ def alloc_host_workspace(prob: FcklProblem, device) -> torch.Tensor:
 
 
 def fused_kl_fwd_bwd_host(hidden, W, topk_idx, topk_logit, row_mask=None, T=1.0, chunk=0,
-                          workspace=None, out=None, loss_host=None, check=True):
+                          workspace=None, out=None, loss_host=None, check=True, dw_rows=0):
     """Forward + backward from HOST inputs (contiguous CPU tensors; pinned for
     overlapped copies): hidden bf16 [N,H], topk_idx int32 [N,K], topk_logit
     float32 [N,K], row_mask uint8 [N] or None.  W is a CUDA bf16 tensor.  The
@@ -178,7 +182,7 @@ def fused_kl_fwd_bwd_host(hidden, W, topk_idx, topk_logit, row_mask=None, T=1.0,
         raise ValueError("W must be a contiguous CUDA tensor")
     if topk_idx.dtype != torch.int32 or topk_logit.dtype != torch.float32:
         raise TypeError("topk_idx must be int32 and topk_logit float32")
-    prob = make_problem(hidden, W, topk_idx, T, chunk)
+    prob = make_problem(hidden, W, topk_idx, T, chunk, dw_rows=dw_rows)
     dev = W.device
     if workspace is None:
         workspace = alloc_host_workspace(prob, dev)
@@ -297,12 +301,12 @@ def select_top_rows(score, n_select, row_mask=None):
 
 
 def fused_kl_rows(hidden, W, topk_idx, topk_logit, rows, T=1.0, chunk=0, workspace=None,
-                  grads=True, want_row_loss=False, check=True, teacher=0):
+                  grads=True, want_row_loss=False, check=True, teacher=0, dw_rows=0):
     """Loss (and dH, dW) over the listed rows only.  Returns (loss, row_loss, dH, dW)."""
     from . import fckl_fwd_bwd_rows
     hidden, W = _bits(hidden), _bits(W)
     _check_inputs(hidden, W, topk_idx, topk_logit, None)
-    prob = make_problem(hidden, W, topk_idx, T, chunk, teacher)
+    prob = make_problem(hidden, W, topk_idx, T, chunk, teacher, dw_rows=dw_rows)
     dev = hidden.device
     if workspace is None:
         workspace = alloc_workspace(prob, dev)

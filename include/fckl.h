@@ -85,11 +85,16 @@ typedef enum {
 
 /* Problem description.  chunk = rows per chunk (0 = automatic: the largest
  * multiple of 128 rows whose bf16 dlogits block [chunk, V] fits in 1 GiB,
- * capped at N rounded up to 64).  The dW GEMM runs once per group of
- * ceil(4096 / chunk) consecutive chunks (at most all of them), so that each
- * read-modify-write of dW covers at least 4096 rows; the workspace holds that
- * group's bf16 dlogits.  Live device bytes are O(max(chunk, 4096) * V) for the
- * workspace plus the caller's O(V * H) weights and gradients. */
+ * capped at N rounded up to 64).  Every chunk runs its own dW GEMM by
+ * default, so the workspace holds one chunk's bf16 dlogits and the live
+ * device bytes are O(chunk * V) of workspace plus the caller's O(N * H)
+ * activations and gradients and O(V * H) weights and dW -- the memory bound of
+ * the chunked loss ("[논문리뷰] Efficient Knowledge Distillation for LLMs",
+ * section 3; aibase.it write-up "Knowledge Distillation 비용 줄이기", section
+ * "chunked KL loss가 하는 일").  dw_rows > chunk groups ceil(dw_rows / chunk)
+ * consecutive chunks into one dW GEMM (at most all of them): fewer
+ * read-modify-writes of the fp32 dW (V * H * 8 bytes each) for small chunks,
+ * at the price of a workspace holding the whole group's dlogits. */
 typedef struct {
   int64_t N;        /* rows (batch * sequence)                  */
   int64_t H;        /* hidden size                              */
@@ -102,6 +107,9 @@ typedef struct {
                             > 0: N_v used for the mean and the gradient
                             scale, e.g. the valid rows of all data-parallel
                             ranks, each rank passing its own row shard */
+  int64_t dw_rows;  /* 0: one dW GEMM per chunk; > 0: each dW GEMM
+                       reduces over at least this many rows (chunks
+                       grouped; see above).  0 <= dw_rows <= INT32_MAX */
 } fckl_problem;
 
 /* What the teacher cache holds in topk_logit [N, K]:
@@ -119,10 +127,10 @@ typedef enum { FCKL_TEACHER_LOGITS = 0, FCKL_TEACHER_PROBS = 1 } fckl_teacher_fo
 
 /* Bytes of device workspace fckl_fwd / fckl_fwd_bwd / fckl_fwd_bwd_rows /
  * fckl_student_entropy need for `prob` (0 when the problem is invalid): the
- * per-chunk teacher, log-sum-exp and dlogits buffers, N floats of row loss,
- * N int32 of compacted row list and the staging buffers that row-list and
- * masked calls gather into.  Pure host arithmetic;
- * needs no GPU. */
+ * per-chunk teacher and log-sum-exp buffers, the bf16 dlogits of one chunk
+ * (of one dW group when dw_rows groups chunks), N floats of row loss, N int32
+ * of compacted row list and the staging buffers that row-list and masked
+ * calls gather into.  Pure host arithmetic; needs no GPU. */
 size_t fckl_workspace_bytes(const fckl_problem* prob);
 
 /* The chunk size the library will use for `prob` (resolves chunk = 0), or -1
@@ -216,10 +224,11 @@ fckl_status fckl_fwd_bwd_host(const fckl_problem* prob, const void* hidden_host,
  *     the device current (one cudaGetSymbolAddress per device); make that
  *     first call before any stream capture on the device.
  *   - The scratch holds N floats of per-row loss plus the per-chunk teacher
- *     and log-sum-exp buffers.  prob->chunk = 0 picks the largest multiple of
- *     256 rows (or N) that fits; an explicit chunk that does not fit, or a
- *     problem for which even 256 rows do not fit, returns FCKL_ERR_WORKSPACE
- *     before anything is enqueued.
+ *     and log-sum-exp buffers.  With prob->chunk = 0 the call takes the
+ *     automatic chunk (see fckl_problem) if its scratch fits, else the largest
+ *     multiple of 256 rows below it whose scratch fits; an explicit chunk that
+ *     does not fit, or a problem for which even 256 rows do not fit, returns
+ *     FCKL_ERR_WORKSPACE before anything is enqueued.
  *   - All calls share the one array and each call re-initialises what must
  *     start at zero; calls that can overlap on the GPU (other streams, other
  *     host threads) race on it and must be serialised by the caller.

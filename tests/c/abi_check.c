@@ -22,7 +22,7 @@ int main(void) {
   fckl_problem p;
   memset(&p, 0, sizeof p);
   p.N = 8192; p.H = 3072; p.V = 128256; p.K = 100; p.T = 1.0f; p.chunk = 0;
-  p.teacher = FCKL_TEACHER_LOGITS; p.n_valid_total = 0;
+  p.teacher = FCKL_TEACHER_LOGITS; p.n_valid_total = 0; p.dw_rows = 0;
 
   CHECK(fckl_resolved_chunk(&p) == 4096);
   size_t ws = fckl_workspace_bytes(&p);
@@ -31,12 +31,23 @@ int main(void) {
   CHECK(strcmp(fckl_status_string(FCKL_OK), "FCKL_OK") == 0);
   CHECK(strcmp(fckl_status_string(FCKL_ERR_WORKSPACE), "FCKL_ERR_WORKSPACE") == 0);
 
+  /* An explicit chunk bounds the dlogits workspace; dw_rows groups chunks. */
+  fckl_problem c = p;
+  c.chunk = 1024;
+  size_t ws1 = fckl_workspace_bytes(&c);
+  CHECK(ws1 >= (size_t)1024 * 128256 * 2 && ws1 < (size_t)1024 * 128256 * 2 + (64u << 20));
+  c.dw_rows = 4096;
+  CHECK(fckl_workspace_bytes(&c) >= ws1 + (size_t)3 * 1024 * 128256 * 2);
+
   fckl_problem bad = p;
   bad.T = NAN;
   CHECK(fckl_workspace_bytes(&bad) == 0);
   CHECK(fckl_resolved_chunk(&bad) == -1);
   bad = p;
   bad.K = FCKL_K_MAX + 1;
+  CHECK(fckl_workspace_bytes(&bad) == 0);
+  bad = p;
+  bad.dw_rows = -1;
   CHECK(fckl_workspace_bytes(&bad) == 0);
 
   /* Host-side rejections happen before any device work. */

@@ -60,13 +60,49 @@ def test_workspace_and_chunk_rules():
     a = fk.fckl_workspace_bytes(FcklProblem(32768, 4096, 128256, 100, 1.0, 1024))
     b = fk.fckl_workspace_bytes(FcklProblem(65536, 4096, 128256, 100, 1.0, 1024))
     assert b - a == 32768 * 8    # only the per-row loss and the compacted row list grow
-    # chunk 1024 < 4096: four chunks of dlogits feed one dW GEMM
-    assert 4 * 1024 * 128256 * 2 <= a < 1100 * 2**20
+    # an explicit chunk bounds the dlogits block: one chunk of bf16 dlogits
+    assert 1024 * 128256 * 2 <= a < 1024 * 128256 * 2 + 48 * 2**20
+    # dw_rows = 4096 groups four 1024-row chunks into one dW GEMM
+    g = fk.fckl_workspace_bytes(FcklProblem(32768, 4096, 128256, 100, 1.0, 1024, dw_rows=4096))
+    assert g - a >= 3 * 1024 * 128256 * 2 + 3 * 1024 * 4096 * 2
+
+
+def test_bench_restates_the_chunk_rule():
+    """bench.py's oracle arm labels its workload with the library's chunk
+    without loading the library; its restatement must agree with it."""
+    import dataclasses
+
+    import bench
+    import synth
+    cases = list(synth.CONFIGS.values())
+    for N, V, chunk in [(100, 4096, 0), (5000, 1000, 0), (70000, 301, 0), (300, 700, 100),
+                        (64, 512, 4096), (1, 64, 0), (1000000, 262144, 0)]:
+        cases.append(dataclasses.replace(synth.CONFIGS[0], N=N, V=V, chunk=chunk))
+    for cfg in cases:
+        want = fk.fckl_resolved_chunk(FcklProblem(cfg.N, cfg.H, cfg.V, cfg.K, cfg.T, cfg.chunk))
+        assert bench.library_chunk(cfg) == want, cfg
+
+
+def test_workspace_follows_an_explicit_chunk():
+    """Live workspace is O(chunk * V): at the gpt-oss shape (V = 201,088) a
+    256-row chunk needs its 256 x V bf16 dlogits block plus small per-chunk
+    buffers and 8 bytes per row (row loss, compacted row list)."""
+    N, H, V, K = 131072, 2880, 201088, 100
+    Vp = (V + 63) // 64 * 64
+    small = fk.fckl_workspace_bytes(FcklProblem(N, H, V, K, 1.0, 256))
+    assert 256 * Vp * 2 + N * 8 <= small < 256 * Vp * 2 + N * 8 + 8 * 2**20
+    big = fk.fckl_workspace_bytes(FcklProblem(N, H, V, K, 1.0, 2048))
+    assert big - small >= (2048 - 256) * Vp * 2
+    # linear in the chunk beyond the per-row arrays
+    mid = fk.fckl_workspace_bytes(FcklProblem(N, H, V, K, 1.0, 1024))
+    assert abs((big - mid) - (mid - small) * 1024 / 768) < 2**20
+    assert fk.fckl_workspace_bytes(FcklProblem(N, H, V, K, 1.0, 256, dw_rows=-1)) == 0
 
 
 @pytest.mark.parametrize("bad", [
     dict(N=0), dict(H=0), dict(V=0), dict(K=0), dict(T=0.0), dict(T=-1.0),
-    dict(T=float("nan")), dict(T=float("inf")), dict(chunk=-1), dict(teacher=2), dict(teacher=-1)])
+    dict(T=float("nan")), dict(T=float("inf")), dict(chunk=-1), dict(teacher=2), dict(teacher=-1),
+    dict(dw_rows=-1)])
 def test_invalid_problem_rejected(bad):
     kw = dict(N=64, H=64, V=512, K=8, T=1.0, chunk=0)
     kw.update(bad)

@@ -30,7 +30,7 @@ def rel_fro(a, b):
     return np.linalg.norm(a - b) / nb if nb > 0 else np.linalg.norm(a)
 
 
-def run_gpu(inp, chunk=None, T=None, fwd_only=False, row_loss=True):
+def run_gpu(inp, chunk=None, T=None, fwd_only=False, row_loss=True, dw_rows=0):
     d = arrays_to_device(inp.hidden, inp.W, inp.topk_idx, inp.topk_logit, inp.row_mask)
     T = inp.cfg.T if T is None else T
     chunk = inp.cfg.chunk if chunk is None else chunk
@@ -38,7 +38,8 @@ def run_gpu(inp, chunk=None, T=None, fwd_only=False, row_loss=True):
         loss, rl = fused_kl_fwd(*d, T=T, chunk=chunk, want_row_loss=row_loss)
         torch.cuda.synchronize()
         return dict(loss=loss.item(), row_loss=rl.cpu().numpy())
-    loss, rl, dH, dW = fused_kl_fwd_bwd(*d, T=T, chunk=chunk, want_row_loss=row_loss)
+    loss, rl, dH, dW = fused_kl_fwd_bwd(*d, T=T, chunk=chunk, want_row_loss=row_loss,
+                                        dw_rows=dw_rows)
     torch.cuda.synchronize()
     return dict(loss=loss.item(), row_loss=rl.cpu().numpy(), dH=dH, dW=dW)
 
@@ -62,12 +63,14 @@ def test_tiny_config_full():
     assert eh < 5e-3 and ew < 5e-3, (eh, ew)   # far inside the stated bound
 
 
-@pytest.mark.parametrize("chunk", [64, 100, 128, 256, 0])
-def test_tiny_config_chunk_invariance(chunk):
-    """Chunking rows differently gives the same loss and gradients."""
+@pytest.mark.parametrize("chunk,dw_rows", [(64, 0), (100, 0), (128, 0), (256, 0), (0, 0),
+                                           (64, 256), (100, 200), (37, 4096)])
+def test_tiny_config_chunk_invariance(chunk, dw_rows):
+    """Chunking rows differently, and grouping chunks into one dW GEMM, gives
+    the same loss and gradients."""
     inp = synth.make_inputs(0)
     ref = run_gpu(inp, chunk=256)
-    g = run_gpu(inp, chunk=chunk)
+    g = run_gpu(inp, chunk=chunk, dw_rows=dw_rows)
     assert abs(g["loss"] - ref["loss"]) <= 1e-5 * abs(ref["loss"])
     np.testing.assert_allclose(g["row_loss"], ref["row_loss"], rtol=1e-5, atol=1e-6)
     assert rel_fro(g["dH"].cpu().numpy(), ref["dH"].cpu().numpy()) < 1e-5
@@ -140,19 +143,22 @@ def _with_valid_count(inp, n_valid, seed):
 
 @pytest.mark.parametrize("n_valid", [1, 63, 100, 150, 190, 299])
 @pytest.mark.parametrize("fill", [0x00, 0xFF])
-def test_compacted_rows_against_oracle(n_valid, fill):
+@pytest.mark.parametrize("dw_rows", [0, 300])
+def test_compacted_rows_against_oracle(n_valid, fill, dw_rows):
     """Masked calls compact their valid rows on the device.  Chunk 100 (not a
-    multiple of 64) with three chunks per dW group puts the partial 64-row block
-    of the dW reduction across chunk slots for some counts; a workspace filled
-    with 0xFF bytes (NaN in bf16 and fp32) shows that no stale value leaks in."""
+    multiple of 64), alone or with three chunks per dW group (dw_rows = 300,
+    which puts the partial 64-row block of the dW reduction across chunk slots
+    for some counts); a workspace filled with 0xFF bytes (NaN in bf16 and fp32)
+    shows that no stale value leaks in."""
     inp = _with_valid_count(synth.make_custom(300, 64, 700, 9, T=1.2, sigma=2.0, seed=21,
                                               chunk=100), n_valid, n_valid)
     o = oracle.oracle_from_inputs(inp)
     d = arrays_to_device(inp.hidden, inp.W, inp.topk_idx, inp.topk_logit, inp.row_mask)
-    prob = FcklProblem(300, 64, 700, 9, 1.2, 100)
+    prob = FcklProblem(300, 64, 700, 9, 1.2, 100, dw_rows=dw_rows)
     ws = alloc_workspace(prob, d[0].device)
     ws.fill_(fill)
-    loss, rl, dH, dW = fused_kl_fwd_bwd(*d, T=1.2, chunk=100, workspace=ws, want_row_loss=True)
+    loss, rl, dH, dW = fused_kl_fwd_bwd(*d, T=1.2, chunk=100, workspace=ws, want_row_loss=True,
+                                        dw_rows=dw_rows)
     torch.cuda.synchronize()
     check_full(inp, dict(loss=loss.item(), row_loss=rl.cpu().numpy(), dH=dH, dW=dW), o)
     ws.fill_(fill)
@@ -171,9 +177,15 @@ def test_llama_8k_config_full():
 
 @pytest.mark.parametrize("cfg", [2, 3, 4])
 def test_large_config_sampled_rows(cfg):
-    """Full-size configs: per-row loss and dH on 64 seeded valid rows against
-    the oracle; the mean of the row losses, the zero column sums of dW and the
-    zero dH of masked rows at full size."""
+    """Full-size configs.  The whole-batch call: per-row loss and dH on 64
+    seeded valid rows against the oracle; the mean of the row losses, the zero
+    column sums of dW and the zero dH of masked rows at full size.  Then the
+    same 64 rows through the listed-row entry point, whose loss, dH rows and
+    full [V, H] dW (the 64 rows' contribution, N_v = 64) the oracle gives
+    exactly: at the workload's own chunk (one 64-row chunk) and in 16-row
+    chunks grouped four to a dW GEMM (dw_rows = 64), so the full-width dW
+    GEMM, the gpt-oss H = 2880 narrow last tile, T = 2 and a grouped dW
+    reduction are all compared with the oracle at the real H and V."""
     inp = synth.make_inputs(cfg)
     rows = synth.sample_rows(inp, 64)
     g = run_gpu(inp)
@@ -193,6 +205,26 @@ def test_large_config_sampled_rows(cfg):
     assert (colsum.abs() <= 2e-2 * scale + 1e-30).all().item()
     del g, dW
     torch.cuda.empty_cache()
+
+    # listed rows: exact oracle targets for loss, dH and dW (N_v = 64)
+    from chunked_kl_loss_tcgen05_b200.torch_api import fused_kl_rows
+    o = oracle.fused_chunked_kl(inp.hidden, inp.W, inp.topk_idx, inp.topk_logit, None,
+                                inp.cfg.T, rows=rows, n_valid=rows.size)
+    o_loss = o["row_loss_rows"].sum() / rows.size
+    d = arrays_to_device(inp.hidden, inp.W, inp.topk_idx, inp.topk_logit, None)
+    rows_d = torch.from_numpy(rows.astype(np.int32)).cuda()
+    for chunk, dw_rows in ((inp.cfg.chunk, 0), (16, 64)):
+        loss, rl, dH, dW = fused_kl_rows(d[0], d[1], d[2], d[3], rows_d, T=inp.cfg.T,
+                                         chunk=chunk, dw_rows=dw_rows, want_row_loss=True)
+        torch.cuda.synchronize()
+        assert abs(loss.item() - o_loss) <= LOSS_RTOL * abs(o_loss), (chunk, loss.item(), o_loss)
+        np.testing.assert_allclose(rl[rows_d].cpu().numpy(), o["row_loss_rows"], rtol=LOSS_RTOL,
+                                   atol=1e-4)
+        eh = rel_fro(dH[rows_d].cpu().numpy(), o["dH_rows"])
+        ew = rel_fro(dW.cpu().numpy(), o["dW"])
+        assert eh <= GRAD_RTOL and ew <= GRAD_RTOL, (chunk, eh, ew)
+        del loss, rl, dH, dW
+        torch.cuda.empty_cache()
 
 
 def _raw_call(inp, ids=None, logits=None):
@@ -346,7 +378,9 @@ def test_sliced_dw_matches_plain_call(n_slices):
 
 
 def test_dp_wrapper_single_rank_nccl():
-    """The data-parallel wrapper on one NCCL rank equals the plain call."""
+    """The data-parallel wrapper on one NCCL rank (valid-count all-reduce, the
+    last dW GEMM in vocabulary slices all-reduced as they finish, loss
+    all-reduce) against the oracle and the plain call."""
     import torch.distributed as dist
     from chunked_kl_loss_tcgen05_b200.dp import fused_kl_fwd_bwd_dp
     import socket
@@ -358,13 +392,48 @@ def test_dp_wrapper_single_rank_nccl():
         inp = synth.make_custom(300, 128, 2000, 10, mask_frac=0.1, seed=82, chunk=128)
         d = arrays_to_device(inp.hidden, inp.W, inp.topk_idx, inp.topk_logit, inp.row_mask)
         l1, _, dH1, dW1 = fused_kl_fwd_bwd(*d, chunk=128)
-        l2, dH2, dW2 = fused_kl_fwd_bwd_dp(*d, chunk=128)
+        l2, dH2, dW2 = fused_kl_fwd_bwd_dp(*d, chunk=128, n_slices=5)
         torch.cuda.synchronize()
         assert l2.item() == pytest.approx(l1.item(), rel=1e-6)
         assert rel_fro(dW2.cpu().numpy(), dW1.cpu().numpy()) < 1e-6
         assert rel_fro(dH2.cpu().numpy(), dH1.cpu().numpy()) < 1e-6
+        o = oracle.oracle_from_inputs(inp)
+        check_full(inp, dict(loss=l2.item(), row_loss=o["row_loss"], dH=dH2, dW=dW2), o)
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("n_shards", [2, 3])
+def test_row_shards_with_global_count_match_oracle(n_shards):
+    """The arithmetic of row-sharded data parallelism on one GPU: each shard of
+    rows runs the sliced fused call with n_valid_total = the valid rows of ALL
+    shards (about n_shards times its own count); the shards' losses and dW
+    partials summed, and their dH rows side by side, equal the oracle on the
+    whole batch (what the all-reduces of the multi-GPU wrapper produce)."""
+    from chunked_kl_loss_tcgen05_b200.dp import shard_rows
+    from chunked_kl_loss_tcgen05_b200.torch_api import fused_kl_fwd_bwd_sliced
+    inp = synth.make_custom(700, 192, 3000, 12, T=1.3, mask_frac=0.15, seed=84, chunk=128)
+    d = arrays_to_device(inp.hidden, inp.W, inp.topk_idx, inp.topk_logit, inp.row_mask)
+    n_total = int((inp.row_mask != 0).sum())
+    loss = 0.0
+    dW = torch.zeros(inp.cfg.V, inp.cfg.H, device="cuda", dtype=torch.float64)
+    dH = torch.empty(inp.cfg.N, inp.cfg.H, device="cuda")
+    for r in range(n_shards):
+        lo, hi = shard_rows(inp.cfg.N, r, n_shards)
+        l, dHs, dWs, slices = fused_kl_fwd_bwd_sliced(
+            d[0][lo:hi], d[1], d[2][lo:hi], d[3][lo:hi], d[4][lo:hi], T=1.3, chunk=128,
+            n_slices=4, n_valid_total=n_total)
+        torch.cuda.synchronize()
+        assert all(ev.query() for _, _, ev in slices)
+        loss += l.item()
+        dW += dWs.double()
+        dH[lo:hi] = dHs
+    o = oracle.oracle_from_inputs(inp)
+    assert abs(loss - o["loss"]) <= LOSS_RTOL * abs(o["loss"]), (loss, o["loss"])
+    eh = rel_fro(dH.cpu().numpy(), o["dH"])
+    ew = rel_fro(dW.cpu().numpy(), o["dW"])
+    assert eh <= GRAD_RTOL and ew <= GRAD_RTOL, (eh, ew)
+    assert eh < 5e-3 and ew < 5e-3, (eh, ew)   # far inside the stated bound
 
 
 def test_autograd_wrapper_gradients():

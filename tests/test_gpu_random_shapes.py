@@ -2,7 +2,8 @@
 the 3-D operand maps (H % 64 == 0), the 2-D ones (H % 64 != 0) and the
 half-width last tile (H % 256 <= 128); vocabularies with a padded last 64-column
 chunk; explicit and automatic chunks; masks from none to most rows;
-temperatures from 0.5 to 3."""
+temperatures from 0.5 to 3; each draw once with one dW GEMM per chunk and once
+with chunks grouped into one dW GEMM (dw_rows)."""
 import numpy as np
 import pytest
 
@@ -26,15 +27,20 @@ def _cases(n=24, seed=2024):
         mask = float(rng.choice([0.0, 0.0, 0.1, 0.5, 0.9]))
         T = float(rng.choice([0.5, 1.0, 1.0, 2.0, 3.0]))
         out.append((i, N, H, V, K, chunk, mask, T))
-    return out
+    # the same draws again with chunks grouped into one dW GEMM (dw_rows)
+    for j, c in enumerate(list(out)):
+        out.append((n + j,) + c[1:] + (int(rng.choice([64, 300, 4096])),))
+    return [c if len(c) == 9 else c + (0,) for c in out]
 
 
-@pytest.mark.parametrize("case", _cases(), ids=lambda c: "N%d_H%d_V%d_K%d_c%d_m%.1f" % c[1:7])
+@pytest.mark.parametrize("case", _cases(),
+                         ids=lambda c: "N%d_H%d_V%d_K%d_c%d_m%.1f" % c[1:7] + "_g%d" % c[8])
 def test_random_shape_matches_oracle(case):
-    i, N, H, V, K, chunk, mask, T = case
-    inp = synth.make_custom(N, H, V, K, T=T, sigma=2.0, mask_frac=mask, seed=500 + i, chunk=chunk)
+    i, N, H, V, K, chunk, mask, T, dw_rows = case
+    inp = synth.make_custom(N, H, V, K, T=T, sigma=2.0, mask_frac=mask, seed=500 + i % 24,
+                            chunk=chunk)
     o = oracle.oracle_from_inputs(inp)
-    g = run_gpu(inp)
+    g = run_gpu(inp, dw_rows=dw_rows)
     if o["n_valid"] == 0:
         assert g["loss"] == 0.0 and not g["dH"].any().item() and not g["dW"].any().item()
         return
