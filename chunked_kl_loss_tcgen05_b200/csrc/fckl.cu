@@ -9,6 +9,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #include "fckl.h"
@@ -223,6 +224,45 @@ int debug_skip_commit() {
   const char* s = std::getenv("FCKL_DEBUG_SKIP_ARRIVE");
   return (s && std::atoi(s) > 0) ? 1 : 0;
 }
+// Tile order of the dH GEMM's split-K units (SchedArgs::tile_order; default 2,
+// chosen on the device; FCKL_DH_ORDER = 0 or 1 fixes it, for measurements).
+int dh_tile_order() {
+  const char* s = std::getenv("FCKL_DH_ORDER");
+  const int v = s ? std::atoi(s) : 2;
+  return (v == 0 || v == 1) ? v : 2;
+}
+// Serpentine k order of the dH GEMM's split-K units (FCKL_DH_SERPENTINE=0
+// turns it off, for measurements).
+int dh_serpentine() {
+  const char* s = std::getenv("FCKL_DH_SERPENTINE");
+  return (s && std::atoi(s) == 0) ? 0 : 1;
+}
+// Programmatic dependent launch for the kernels of a call (FCKL_NO_PDL=1 turns
+// it off: every kernel then starts after the previous one has completed).
+bool pdl_enabled() {
+  const char* s = std::getenv("FCKL_NO_PDL");
+  return !(s && std::atoi(s) > 0);
+}
+
+// Launches `kernel` on `st`, with programmatic stream serialization when
+// `pdl`: the kernel may start once every CTA of the previous kernel has
+// called pdl_trigger() (or exited); it calls pdl_wait() before it touches what
+// that kernel produces.  Kernels with compile-time cluster dimensions keep them.
+template <typename... KArgs, typename... Args>
+cudaError_t launch(bool pdl, void (*kernel)(KArgs...), int grid, int block, size_t smem,
+                   cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3((unsigned)block, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // ---------------------------------------------------------------- profiling
 enum Kind {
@@ -389,6 +429,14 @@ fckl_status run(const Request& q) {
   const float invT = 1.0f / prob->T;
   const float scale2 = 1.4426950408889634f / prob->T;
   CtlArgs ca{ctl, wait_timeout_ns(), debug_skip_commit()};
+  const bool pdl = pdl_enabled();
+  // Launch with programmatic dependent launch; a failed launch ends the call.
+#define FCKL_LAUNCH(kernel, grid, block, smem, ...)                                   \
+  do {                                                                                 \
+    if (launch(pdl, kernel, (int)(grid), (int)(block), (size_t)(smem), st, __VA_ARGS__) != \
+        cudaSuccess)                                                                   \
+      return FCKL_ERR_CUDA;                                                            \
+  } while (0)
 
   if (cudaMemsetAsync(ctl, 0, sizeof(DeviceCtl), st) != cudaSuccess) return FCKL_ERR_CUDA;
   if (q.ready && cudaStreamWaitEvent(st, q.ready[0], 0) != cudaSuccess) return FCKL_ERR_CUDA;
@@ -396,11 +444,14 @@ fckl_status run(const Request& q) {
     ProfScope ps(K_COUNT, st, 0.0,
                  user_list ? q.n_rows * 4.0 : (q.row_mask ? L.N * (compact ? 5.0 : 1.0) : 0.0));
     if (user_list)
-      k_count_list<<<1, 1024, 0, st>>>(q.rows, q.n_rows, L.N, (int)prob->n_valid_total, ctl);
+      FCKL_LAUNCH(k_count_list, 1, 1024, 0, q.rows, (long long)q.n_rows, (long long)L.N,
+                  (int)prob->n_valid_total, ctl);
     else if (compact)
-      k_compact_mask<<<1, 1024, 0, st>>>(q.row_mask, L.N, (int)prob->n_valid_total, clist, ctl);
+      FCKL_LAUNCH(k_compact_mask, 1, 1024, 0, q.row_mask, (long long)L.N,
+                  (int)prob->n_valid_total, clist, ctl);
     else
-      k_count_valid<<<1, 1024, 0, st>>>(q.row_mask, L.N, (int)prob->n_valid_total, ctl);
+      FCKL_LAUNCH(k_count_valid, 1, 1024, 0, q.row_mask, (long long)L.N,
+                  (int)prob->n_valid_total, ctl);
   }
   // The profiler's flop and byte counts follow the rows a launch really
   // processes; for a compacted call it reads their number back once (profiling
@@ -466,11 +517,11 @@ fckl_status run(const Request& q) {
       __nv_bfloat16* hdst = hstage + (size_t)(c % G) * L.C * L.H;
       {
         ProfScope ps(K_GATHER, st, 0.0, nr * (L.H * 4.0 + K * 16.0 + 5.0));
-        k_gather_rows<<<cap, 128, 0, st>>>(
-            rowlist + row0, rc, L.N, H, K, static_cast<const __nv_bfloat16*>(q.hidden),
-            q.topk_idx, q.topk_logit, hdst, idstage, lgstage, mstage,
-            bwd ? reinterpret_cast<uint4*>(dlog + (size_t)(c % G) * L.C * L.Vp) : nullptr,
-            L.Vp / 8);
+        FCKL_LAUNCH(k_gather_rows, cap, 128, 0, rowlist + row0, rc, (long long)L.N, H, K,
+                    static_cast<const __nv_bfloat16*>(q.hidden), q.topk_idx, q.topk_logit, hdst,
+                    idstage, lgstage, mstage,
+                    bwd ? reinterpret_cast<uint4*>(dlog + (size_t)(c % G) * L.C * L.Vp) : nullptr,
+                    (long long)(L.Vp / 8));
       }
       h_c = hdst; ids_c = idstage; lg_c = lgstage; rl_c = rlstage; dH_c = dhstage;
       mask_c = compact ? nullptr : mstage;  // compacted rows are all valid
@@ -496,61 +547,64 @@ fckl_status run(const Request& q) {
       EpiEntropy::Params pe{V, 1, (int)NT, scale2, nullptr, nullptr, nullptr, part, upart};
       {
         ProfScope ps(K_ENT, st, gemm_flops, 2.0 * (nr + (double)L.V) * L.H + nr * NT * 12.0);
-        gemm_pair_kernel<EpiEntropy, false, false>
-            <<<Gv, GEMM_THREADS, pair_smem_bytes<EpiEntropy>(), st>>>(mapH_k, mapW_k, mapW_k, pe,
-                                                                      sa_v, ca);
+        FCKL_LAUNCH((gemm_pair_kernel<EpiEntropy, false, false>), Gv, GEMM_THREADS,
+                    pair_smem_bytes<EpiEntropy>(), mapH_k, mapW_k, mapW_k, pe, sa_v, ca);
       }
       {
         ProfScope ps(K_ENT_MERGE, st, 0.0, nr * NT * 12.0 + nr * 5.0);
-        k_merge_entropy<<<row_blocks, ROW_WARPS * 32, 0, st>>>(part, upart, (int)NT, rc, mask_c,
-                                                               q.entropy + row0);
+        FCKL_LAUNCH(k_merge_entropy, row_blocks, ROW_WARPS * 32, 0, (const float2*)part,
+                    (const float*)upart, (int)NT, rc, mask_c, q.entropy + row0);
       }
       continue;
     }
 
     {
       ProfScope ps(K_PREP, st, 0.0, nr * K * 20.0 + nr * (NT + 1) * 2.0);
-      k_prep_teacher<<<row_blocks, ROW_WARPS * 32, 0, st>>>(
-          ids_c, lg_c, mask_c, rc, K, V, (int)NT, invT, prob->teacher == FCKL_TEACHER_PROBS,
-          sid, sp, zs, tstart, plogp, ctl);
+      // prep also zeroes the chunk's dH rows, into which the dH GEMM reduce-adds
+      FCKL_LAUNCH(k_prep_teacher, row_blocks, ROW_WARPS * 32, 0, ids_c, lg_c, mask_c, rc, K, V,
+                  (int)NT, invT, prob->teacher == FCKL_TEACHER_PROBS, sid, sp, zs, tstart, plogp,
+                  ctl, bwd ? dH_c : (float*)nullptr, H);
     }
     EpiLse::Params pf{V, K, (int)NT, scale2, sid, tstart, zs, part, nullptr};
     CtlArgs ca_f = ca;
     ca_f.debug_skip_commit = (c == 0) ? ca.debug_skip_commit : 0;
     {
       ProfScope ps(K_FWD, st, gemm_flops, 2.0 * (nr + (double)L.V) * L.H + nr * NT * 8.0);
-      gemm_pair_kernel<EpiLse, false, false>
-          <<<Gv, GEMM_THREADS, pair_smem_bytes<EpiLse>(), st>>>(mapH_k, mapW_k, mapW_k, pf, sa_v,
-                                                                ca_f);
+      FCKL_LAUNCH((gemm_pair_kernel<EpiLse, false, false>), Gv, GEMM_THREADS,
+                  pair_smem_bytes<EpiLse>(), mapH_k, mapW_k, mapW_k, pf, sa_v, ca_f);
     }
     {
       ProfScope ps(K_MERGE, st, 0.0, nr * K * 8.0 + nr * NT * 8.0 + nr * 13.0);
-      k_merge_loss<<<row_blocks, ROW_WARPS * 32, 0, st>>>(part, (int)NT, rc, K, invT, zs, sp,
-                                                           plogp, mask_c, lse2, rl_c);
+      FCKL_LAUNCH(k_merge_loss, row_blocks, ROW_WARPS * 32, 0, (const float2*)part, (int)NT, rc,
+                  K, invT, (const float*)zs, (const float*)sp, (const float*)plogp, mask_c, lse2,
+                  rl_c);
     }
     if (!bwd) {
       if (list) {
         ProfScope ps(K_SCATTER, st, 0.0, nr * 12.0);
-        k_scatter_rows<<<cap, 128, 0, st>>>(rowlist + row0, rc, L.N, H, rlstage, rl, nullptr,
-                                            nullptr);
+        FCKL_LAUNCH(k_scatter_rows, cap, 128, 0, rowlist + row0, rc, (long long)L.N, H,
+                    (const float*)rlstage, rl, (const float*)nullptr, (float*)nullptr);
       }
       continue;
     }
 
-    // Backward 1: recompute the tiles and form bf16 dlogits = q - p~.
+    // Backward 1: recompute the tiles and form bf16 dlogits = q - p~.  Its
+    // operands (h, W) were complete before the kernel ahead of it launched, so
+    // its main loop starts at once and only its epilogue waits for the merge.
     EpiDlogits::Params pb{V, K, (int)NT, scale2, lse2, sid, tstart, sp, mask_c};
+    SchedArgs sa_b = sa_v;
+    sa_b.early = 1;
     CUtensorMap mapD_st;
     // The store map spans the padded width: the pad columns receive zeros.
     if (!make_map(&mapD_st, dlog_c, L.Vp, cap, L.Vp * 2, 64, 32)) return FCKL_ERR_CUDA;
     {
       ProfScope ps(K_BWD, st, gemm_flops, 2.0 * (nr + (double)L.V) * L.H + 2.0 * nr * L.V);
-      gemm_pair_kernel<EpiDlogits, false, false>
-          <<<Gv, GEMM_THREADS, pair_smem_bytes<EpiDlogits>(), st>>>(mapH_k, mapW_k, mapD_st, pb,
-                                                                    sa_v, ca);
+      FCKL_LAUNCH((gemm_pair_kernel<EpiDlogits, false, false>), Gv, GEMM_THREADS,
+                  pair_smem_bytes<EpiDlogits>(), mapH_k, mapW_k, mapD_st, pb, sa_b, ca);
     }
 
-    // Backward 2: dH[rows] = alpha * dlogits W; A = dlogits (K-major), B = W (MN-major).
-    if (cudaMemsetAsync(dH_c, 0, (size_t)cap * L.H * 4, st) != cudaSuccess) return FCKL_ERR_CUDA;
+    // Backward 2: dH[rows] = alpha * dlogits W; A = dlogits (K-major), B = W (MN-major),
+    // reduce-added into the rows k_prep_teacher zeroed.
     CUtensorMap mapD_k, mapD_mn, mapH_mn, mapdH;
     if (!make_map(&mapD_k, dlog_c, L.V, cap, L.Vp * 2, BK, CM)) return FCKL_ERR_CUDA;
     if (!make_map(&mapdH, dH_c, L.H, cap, L.H * 4, 32, 32, true)) return FCKL_ERR_CUDA;
@@ -558,18 +612,20 @@ fckl_status run(const Request& q) {
     // A compacted chunk's row count is only known on the device: the kernel
     // picks the split there (S = 0) and the launch covers every pair.
     const int S = compact ? 0 : choose_split(tiles_h, KBv, pairs);
-    SchedArgs sa_h{SCHED_SPLIT_K, (int)NTh, (int)KBv, S, 0, rc, 0, w3d, 0, narrow_h};
+    SchedArgs sa_h{SCHED_SPLIT_K, (int)NTh, (int)KBv, S, 0, rc, 0, w3d, 0, narrow_h, 0,
+                   dh_tile_order(), dh_serpentine()};
     EpiDH::Params ph{H, invT, ctl};
     {
       ProfScope ps(K_DH, st, gemm_flops,
                    2.0 * nr * (double)L.V + 2.0 * (double)L.V * L.H + 4.0 * nr * L.H);
-      gemm_pair_kernel<EpiDH, false, true>
-          <<<S > 0 ? grid_for(tiles_h * S) : 2 * pairs, GEMM_THREADS, pair_smem_bytes<EpiDH>(), st>>>(
-              mapD_k, mapW_mn, mapdH, ph, sa_h, ca);
+      FCKL_LAUNCH((gemm_pair_kernel<EpiDH, false, true>),
+                  S > 0 ? grid_for(tiles_h * S) : 2 * pairs, GEMM_THREADS, pair_smem_bytes<EpiDH>(),
+                  mapD_k, mapW_mn, mapdH, ph, sa_h, ca);
     }
     if (list) {
       ProfScope ps(K_SCATTER, st, 0.0, nr * (12.0 + 8.0 * L.H));
-      k_scatter_rows<<<cap, 128, 0, st>>>(rowlist + row0, rc, L.N, H, rlstage, rl, dhstage, q.dH);
+      FCKL_LAUNCH(k_scatter_rows, cap, 128, 0, rowlist + row0, rc, (long long)L.N, H,
+                  (const float*)rlstage, rl, (const float*)dhstage, q.dH);
     }
 
     // Backward 3, once per group of G chunks (or at the last chunk):
@@ -588,8 +644,8 @@ fckl_status run(const Request& q) {
     EpiDW::Params pw{V, H, invT, g0 > 0 ? 1 : 0, ctl};
     if (compact && g0 == 0) {  // with no valid row no dW launch below writes dW
       ProfScope ps(K_ZERO_DW, st, 0.0, 0.0);
-      k_zero_if_no_valid<<<2 * pairs, 256, 0, st>>>(reinterpret_cast<float4*>(q.dW),
-                                                     L.V * L.H / 4, ctl);
+      FCKL_LAUNCH(k_zero_if_no_valid, 2 * pairs, 256, 0, reinterpret_cast<float4*>(q.dW),
+                  (long long)(L.V * L.H / 4), (const DeviceCtl*)ctl);
     }
     // One launch over all vocabulary tiles, or -- for the last group of a
     // sliced call -- one launch per slice, each followed by its event.
@@ -601,15 +657,16 @@ fckl_status run(const Request& q) {
     for (long long i = 0; i < ns; ++i) {
       const long long mt0 = i * MTv / ns, mt1 = (i + 1) * MTv / ns;
       const long long v0 = mt0 * PM, v1 = std::min<long long>(L.V, mt1 * PM);
+      // The dW main loop reads only dlogits and h, complete before the kernel
+      // ahead of it launched: it starts at once, the epilogue waits.
       SchedArgs sa_w{SCHED_TILES, (int)NTh, 0, 1, (int)(mt1 - mt0), rows_of(grow0, gcap), d3d, h3d,
-                     (int)mt0, narrow_h};
+                     (int)mt0, narrow_h, 1};
       {
         const double vs = (double)(v1 - v0);
         ProfScope ps(K_DW, st, 2.0 * gr * vs * (double)L.H,
                      2.0 * gr * vs + 2.0 * gr * L.H * ns + (g0 > 0 ? 8.0 : 4.0) * vs * L.H);
-        gemm_pair_kernel<EpiDW, true, true>
-            <<<grid_for((mt1 - mt0) * NTh), GEMM_THREADS, pair_smem_bytes<EpiDW>(), st>>>(
-                mapD_mn, mapH_mn, mapdW, pw, sa_w, ca);
+        FCKL_LAUNCH((gemm_pair_kernel<EpiDW, true, true>), grid_for((mt1 - mt0) * NTh),
+                    GEMM_THREADS, pair_smem_bytes<EpiDW>(), mapD_mn, mapH_mn, mapdW, pw, sa_w, ca);
       }
       if (sliced) {
         if (cudaEventRecord(q.slice_events[i], st) != cudaSuccess) return FCKL_ERR_CUDA;
@@ -626,8 +683,10 @@ fckl_status run(const Request& q) {
   }
   if (!ent) {
     ProfScope ps(K_FINAL, st, 0.0, (double)L.N * 4.0);
-    k_finalize<<<1, 1024, 0, st>>>(rl, L.N, ctl, q.loss);
+    FCKL_LAUNCH(k_finalize, 1, 1024, 0, (const float*)rl, (long long)L.N, (const DeviceCtl*)ctl,
+                q.loss);
   }
+#undef FCKL_LAUNCH
   if (cudaGetLastError() != cudaSuccess) return FCKL_ERR_CUDA;
   return FCKL_OK;
 }

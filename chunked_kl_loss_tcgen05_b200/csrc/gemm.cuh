@@ -87,6 +87,7 @@ struct RowCount {
 struct Work {
   int mt, nt;    // pair tile: rows [mt*256, +256), columns [nt*256, +256)
   int kb0, kb1;  // k-blocks [kb0, kb1) of 64
+  int rev;       // 1: walk the k-blocks from kb1 - 1 down to kb0
   int m0, n0;    // this CTA's first row (mt*256 + 128*rank) and the first column
   int rows;      // rows of the launch (row-tiled kernels: rows >= rows are padding)
 };
@@ -111,6 +112,25 @@ struct SchedArgs {
   // 1: the last column tile holds at most 128 columns, so it runs as an
   // N = 128 MMA (each CTA of the pair stages 64 columns of B) instead of 256.
   int narrow_tail;
+  // Programmatic dependent launch.  0: every thread waits for the preceding
+  // kernel before touching global memory, then lets the next kernel launch.
+  // 1: the operands were complete before the preceding kernel launched, so the
+  // producer and the MMA issuer start at once (overlapping the tail of the
+  // kernels before) and only the epilogue waits; the next kernel may launch
+  // right away (it waits for this one before touching memory).
+  int early;
+  // SCHED_SPLIT_K: order of the output tiles inside a k segment.  0: column
+  // tile fastest (the pairs running at once cover few row tiles and every
+  // column tile: A re-read little, B once per wave); 1: row tile fastest (the
+  // reverse); 2: chosen when the kernel starts -- row tile fastest when the
+  // launch's rows are at most its columns, so that the smaller operand is the
+  // one re-read.
+  int tile_order;
+  // SCHED_SPLIT_K: 1 = serpentine k order -- units of odd waves walk their
+  // k segment backwards, so they start on the k-blocks the wave before them
+  // touched last, which are still in L2 (the operand every wave re-reads is
+  // then served mostly from L2 instead of DRAM).
+  int serpentine;
 };
 
 __device__ __forceinline__ bool narrow_unit(const SchedArgs& a, const Work& w) {
@@ -151,6 +171,7 @@ struct PairSched {
       MT = row_tiles; KB = a.KB; tiles = MT * a.NT; total = (long long)tiles;
     } else if (a.kind == SCHED_SPLIT_K) {
       MT = row_tiles; KB = a.KB; tiles = MT * a.NT; total = (long long)tiles * a.S;
+      if (a.tile_order == 2) a.tile_order = rows <= a.NT * BN ? 1 : 0;
     } else {
       MT = a.MT; KB = (rows + BK - 1) / BK; tiles = MT * a.NT;
       total = rows > 0 ? (long long)tiles : 0;
@@ -161,18 +182,23 @@ struct PairSched {
     if (a.kind == SCHED_VOCAB_MAJOR) {
       w.nt = (int)(u / MT);
       w.mt = (int)(u - (long long)w.nt * MT);
-      w.kb0 = 0; w.kb1 = KB;
+      w.kb0 = 0; w.kb1 = KB; w.rev = 0;
     } else if (a.kind == SCHED_SPLIT_K) {
       const int ks = (int)(u / tiles);
       const int tile = (int)(u - (long long)ks * tiles);
-      w.mt = tile / a.NT; w.nt = tile - w.mt * a.NT;
+      if (a.tile_order == 1) {
+        w.nt = tile / MT; w.mt = tile - w.nt * MT;
+      } else {
+        w.mt = tile / a.NT; w.nt = tile - w.mt * a.NT;
+      }
       w.kb0 = (int)((long long)ks * KB / a.S);
       w.kb1 = (int)((long long)(ks + 1) * KB / a.S);
+      w.rev = a.serpentine ? (int)((u / G) & 1) : 0;  // odd waves walk backwards
     } else {
       const int t = (int)(u / a.NT);
       w.nt = (int)(u - (long long)t * a.NT);
       w.mt = a.mt0 + t;
-      w.kb0 = 0; w.kb1 = KB;
+      w.kb0 = 0; w.kb1 = KB; w.rev = 0;
     }
     w.rows = rows;
     u += G;
@@ -245,6 +271,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
   __syncthreads();
   cluster_sync_all();  // barriers of both CTAs initialised before any remote use
   tc_fence_after();
+  if (!sa.early) pdl_wait();
+  pdl_trigger();
   const uint32_t tmem_base = *tmem_slot;
   const WaitCtx wc{ca.timeout_ns, ca.ctl, abort_flag};
 
@@ -261,7 +289,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
       while (ok && sch.next(w)) {
         const int a_row = w.mt * PM + (int)rank * CM;
         const int b_col = w.nt * BN + (int)rank * (narrow_unit(sa, w) ? 64 : BN / 2);
-        for (int kb = w.kb0; kb < w.kb1; ++kb) {
+        for (int i = 0; i < w.kb1 - w.kb0; ++i) {
+          const int kb = w.rev ? w.kb1 - 1 - i : w.kb0 + i;
           if (!wait_phase(smem_u32(&empty[stage]), phase ^ 1u, wc, SITE_PROD_EMPTY)) {
             ok = false;
             break;
@@ -324,7 +353,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
         const uint32_t idesc = narrow_unit(sa, w) ? idesc_narrow : idesc_full;
-        for (int kb = w.kb0; kb < w.kb1; ++kb) {
+        for (int i = 0; i < w.kb1 - w.kb0; ++i) {  // k order is the producer's
           if (!wait_phase(smem_u32(&full[stage]), phase, wc, SITE_MMA_FULL)) {
             ok = false;
             break;
@@ -338,7 +367,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
                                      : sw128_desc(a_base + k * 32, 16, 1024);
             const uint64_t bd = B_MN ? sw128_desc(b_base + k * 2048, 8192, 1024)
                                      : sw128_desc(b_base + k * 32, 16, 1024);
-            umma_bf16_pair(d_tmem, ad, bd, idesc, (kb > w.kb0 || k > 0) ? 1u : 0u);
+            umma_bf16_pair(d_tmem, ad, bd, idesc, (i > 0 || k > 0) ? 1u : 0u);
           }
           umma_commit_pair(smem_u32(&empty[stage]), 0x3);  // frees the stage in both CTAs
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -369,6 +398,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
     Work w;
     int acc = 0;
     uint32_t acc_phase = 0;
+    if (sa.early) pdl_wait();  // the epilogue reads and writes what earlier kernels produce
     typename Epi::State st;
     Epi::init(ep, st, sEpi + quarter * (Epi::kSmemBytes / 4), lane);
     while (sch.next(w)) {

@@ -34,6 +34,21 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// ---------------------------------------------------------------- dependent launch
+// Programmatic dependent launch (kernels launched with programmatic stream
+// serialization).  pdl_wait(): block until the preceding kernel of the stream
+// has completed and its memory operations are visible (a no-op for a kernel
+// launched without the attribute).  pdl_trigger(): allow the next kernel of
+// the stream to launch once every CTA of this grid has triggered or exited.
+// Every kernel of the library calls pdl_wait() before it exits, so the
+// completion of a kernel implies the completion of all kernels before it.
+__device__ __forceinline__ void pdl_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");

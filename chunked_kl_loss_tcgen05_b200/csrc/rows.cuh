@@ -28,6 +28,8 @@ __device__ __forceinline__ float warp_sum(float x) {
 // caller's total (> 0) when the rows are one shard of a larger batch.  One block.
 __global__ void __launch_bounds__(1024) k_count_valid(const uint8_t* __restrict__ mask, long long N,
                                                       int total, DeviceCtl* ctl) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int red[32];
   int c = 0;
   if (mask == nullptr) {
@@ -51,6 +53,8 @@ __global__ void __launch_bounds__(1024) k_count_valid(const uint8_t* __restrict_
 // padding and are skipped; entries >= N are reported as bad indices.  One block.
 __global__ void __launch_bounds__(1024) k_count_list(const int32_t* __restrict__ rows, long long n,
                                                      long long N, int total, DeviceCtl* ctl) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int red[32];
   int c = 0;
   bool bad = false;
@@ -83,6 +87,8 @@ __global__ void __launch_bounds__(1024) k_compact_mask(const uint8_t* __restrict
 // dW = 0 when the call compacted no row (then no dW launch writes it);
 // otherwise nothing.
 __global__ void k_zero_if_no_valid(float4* __restrict__ out, long long n4, const DeviceCtl* ctl) {
+  pdl_trigger();  // the dW GEMM after it may start its main loop
+  pdl_wait();
   if (ctl->n_rows > 0) return;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4;
        i += (long long)gridDim.x * blockDim.x)
@@ -102,6 +108,8 @@ __global__ void __launch_bounds__(128)
                   const float* __restrict__ lg, __nv_bfloat16* __restrict__ hst,
                   int32_t* __restrict__ idst, float* __restrict__ lgst, uint8_t* __restrict__ mst,
                   uint4* __restrict__ dlz, long long dl_u4) {
+  pdl_wait();
+  pdl_trigger();
   const int i = blockIdx.x;
   const int n = rc.get();
   if (i >= n) {
@@ -132,6 +140,8 @@ __global__ void __launch_bounds__(128)
     k_scatter_rows(const int32_t* __restrict__ list, RowCount rc, long long N, int H,
                    const float* __restrict__ rl_stage, float* __restrict__ rl,
                    const float* __restrict__ dh_stage, float* __restrict__ dH) {
+  pdl_trigger();  // the dW GEMM after it may start its main loop
+  pdl_wait();
   const int i = blockIdx.x;
   if (i >= rc.get()) return;
   const int r = list[i];
@@ -179,6 +189,8 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* sh, int* total) 
 __global__ void __launch_bounds__(1024) k_compact_mask(const uint8_t* __restrict__ mask,
                                                        long long N, int total,
                                                        int32_t* __restrict__ list, DeviceCtl* ctl) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ int sh[32];
   const long long per = (N + blockDim.x - 1) / blockDim.x;
   const long long i0 = threadIdx.x * per, i1 = (i0 + per < N) ? i0 + per : N;
@@ -279,19 +291,28 @@ __global__ void __launch_bounds__(1024)
 // of 256 columns the position of its first id in the sorted list (tstart,
 // NT + 1 entries per row), so that a GEMM epilogue finds the cached ids of its
 // tile with one load.  Ids outside [0, V) are recorded as an error and replaced
-// by INT_MAX, which no vocab column matches.
+// by INT_MAX, which no vocab column matches.  When dH_row0 is given, the warp
+// also zeroes its row of dH (H floats), which the chunk's dH GEMM reduce-adds
+// into.
 __global__ void __launch_bounds__(ROW_WARPS * 32)
     k_prep_teacher(const int32_t* __restrict__ ids, const float* __restrict__ lg,
                    const uint8_t* __restrict__ mask, RowCount rc, int K, int V, int NT,
                    float invT, bool probs, int* __restrict__ sid, float* __restrict__ sp,
                    float* __restrict__ zs, uint16_t* __restrict__ tstart,
-                   float* __restrict__ plogp, DeviceCtl* ctl) {
+                   float* __restrict__ plogp, DeviceCtl* ctl, float* __restrict__ dH_row0,
+                   int H) {
   __shared__ int s_ids[ROW_WARPS][K_MAX];
   __shared__ int s_sorted[ROW_WARPS][K_MAX];
   __shared__ float s_sp[ROW_WARPS][K_MAX];
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * ROW_WARPS + warp;
   if (row >= rc.get()) return;  // warp-uniform
+  if (dH_row0 != nullptr) {  // the dH GEMM of this chunk reduce-adds into zeroed rows
+    float4* z = reinterpret_cast<float4*>(dH_row0 + (size_t)row * H);
+    for (int j = lane; j < H / 4; j += 32) z[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   const bool keep = mask == nullptr || mask[row] != 0;
   float t[K_MAX / 32];
   int id[K_MAX / 32];
@@ -395,6 +416,8 @@ __global__ void __launch_bounds__(ROW_WARPS * 32)
                  const float* __restrict__ zs, const float* __restrict__ sp,
                  const float* __restrict__ plogp, const uint8_t* __restrict__ mask,
                  float* __restrict__ lse2_out, float* __restrict__ row_loss) {
+  pdl_trigger();  // the recompute GEMM after it may start its main loop
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * ROW_WARPS + warp;
   if (row >= rc.get()) return;
@@ -430,6 +453,8 @@ __global__ void __launch_bounds__(ROW_WARPS * 32)
 __global__ void __launch_bounds__(ROW_WARPS * 32)
     k_merge_entropy(const float2* __restrict__ partials, const float* __restrict__ upart, int NT,
                     RowCount rc, const uint8_t* __restrict__ mask, float* __restrict__ entropy) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * ROW_WARPS + warp;
   if (row >= rc.get()) return;
@@ -458,6 +483,8 @@ __global__ void __launch_bounds__(ROW_WARPS * 32)
 // loss = sum(row_loss) / N_valid, fp64 accumulation in a fixed order.
 __global__ void __launch_bounds__(1024) k_finalize(const float* __restrict__ row_loss, long long N,
                                                    const DeviceCtl* ctl, float* loss) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ double red[1024];
   double s = 0.0;
   for (long long i = threadIdx.x; i < N; i += blockDim.x) s += (double)row_loss[i];
