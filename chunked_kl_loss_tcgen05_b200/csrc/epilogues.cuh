@@ -7,9 +7,10 @@
 //               gather of z at the row's cached teacher ids that fall in the
 //               tile.  Nothing of the tile is written; one (max, sum) partial
 //               per row per vocab tile.
-//   EpiDlogits  backward: recomputed z tile -> q - p~ (0 for masked rows and
-//               for columns >= V), rounded once to bf16, staged in shared
-//               memory and TMA-stored to the chunk's dlogits block.
+//   EpiDlogits  backward: recomputed z tile -> q - p~ (0 for masked rows,
+//               for rows past the launch's rows and for columns >= V),
+//               rounded once to bf16, staged in shared memory and
+//               TMA-stored to the chunk's dlogits block.
 //   EpiDH       dH[rows, :] += alpha * (dlogits W) partial (split-K): fp32
 //               tile staged in shared memory, TMA reduce-add into dH.
 //   EpiDW       dW (+)= alpha * (dlogits^T h): TMA store (first chunk) or
@@ -151,6 +152,7 @@ struct EpiDlogits {
     const uint16_t* tstart;   // [rows_c, NT + 1] first sorted position of each vocab tile
     const float* sp;          // [rows_c, K] teacher probabilities, same order
     const uint8_t* mask;      // chunk rows, or nullptr
+    int store_rows;           // rows of the store map (the chunk's row capacity)
   };
   struct State {
     int cur, nid, n;
@@ -195,6 +197,10 @@ struct EpiDlogits {
     const float lse = keep ? p.lse2[row] : 0.f;
     const int col0 = w.n0;
     const int y = w.m0 + quarter * 32;
+    // Slabs of 32 rows are stored up to the launch's rows rounded up to 64
+    // (rows past the last row hold zeros: the dW GEMM reads whole 64-row
+    // blocks), never starting outside the store map.
+    const int y_end = min((w.rows + 63) & ~63, p.store_rows);
     st.nid = INT_MAX;
     if (keep) {
       st.cur = __ldg(p.tstart + (size_t)row * (p.NT + 1) + w.nt);
@@ -224,7 +230,7 @@ struct EpiDlogits {
                                                     pack_bf16x2(v1[8 * j + 6], v1[8 * j + 7]));
       stage_release();
       if (lane == 0) {  // one group per slice, empty when the slice lies outside the map
-        if (base < p.V && y < w.rows) tma_store_2d(mapC, smem_u32(buf), base, y);
+        if (base < p.V && y < y_end) tma_store_2d(mapC, smem_u32(buf), base, y);
         bulk_commit();
       }
       ++st.n;

@@ -97,7 +97,8 @@ Layout make_layout(const fckl_problem* p, bool full = true) {
   L.off_part = take(C * L.NT * sizeof(float2));
   L.off_upart = take(full ? C * L.NT * 4 : 0);
   // Row-list calls gather their rows into these staging buffers.
-  L.off_hstage = take(full ? (size_t)L.G * C * L.H * 2 : 0);
+  // two buffers of a group's gathered hidden rows (alternating by group)
+  L.off_hstage = take(full ? 2 * (size_t)L.G * C * L.H * 2 : 0);
   L.off_idstage = take(full ? C * L.K * 4 : 0);
   L.off_lgstage = take(full ? C * L.K * 4 : 0);
   L.off_mstage = take(full ? C : 0);
@@ -495,95 +496,138 @@ fckl_status run(const Request& q) {
   auto rows_of = [&](long long row0, long long cap) {
     return compact ? RowCount{-1, ctl, (int)row0, (int)cap} : RowCount{(int)cap, ctl, 0, 0};
   };
-  for (long long c = 0; c < nchunks; ++c) {
-    if (q.ready && cudaStreamWaitEvent(st, q.ready[1 + c], 0) != cudaSuccess) return FCKL_ERR_CUDA;
-    const long long row0 = c * L.C;
-    const int cap = (int)std::min(L.C, R - row0);  // rows of the chunk (upper bound if compact)
-    const RowCount rc = rows_of(row0, cap);
-    // rows this chunk processes, as far as the host knows (profiling figures)
-    const double nr = prof_rows < 0 ? (double)cap
-                                    : (double)std::max(0LL, std::min<long long>(cap, prof_rows - row0));
-    const long long MT = cdiv(cap, PM);
-    const int row_blocks = (int)cdiv(cap, ROW_WARPS);
-    // Sources and destinations of this chunk: the caller's rows directly, or
-    // the staging buffers the listed / compacted rows are gathered into.
-    const void* h_c;
-    const int32_t* ids_c;
-    const float* lg_c;
-    const uint8_t* mask_c;
-    float* rl_c;
-    float* dH_c;
+  // One chunk's rows and where they come from: the caller's rows directly,
+  // or the staging buffers the listed / compacted rows are gathered into.
+  // Staged hidden rows alternate between two buffers (by dW group), so that
+  // the next chunk can be gathered while the current group's dW GEMM still
+  // reads its rows.
+  struct ChunkIO {
+    long long row0;
+    int cap;              // rows of the chunk (upper bound if compact)
+    RowCount rc;
+    double nr;            // rows processed, as far as the host knows (profiling figures)
+    long long MT;
+    int row_blocks;
+    const void* h;
+    const int32_t* ids;
+    const float* lg;
+    const uint8_t* mask;
+    float* rl;
+    float* dH;
+    __nv_bfloat16* dlog;  // this chunk's rows in the group's dlogits block
+  };
+  auto hslot = [&](long long c) {
+    return hstage + (size_t)(((c / G) & 1) * G + c % G) * L.C * L.H;
+  };
+  auto chunk_io = [&](long long c) {
+    ChunkIO io;
+    io.row0 = c * L.C;
+    io.cap = (int)std::min(L.C, R - io.row0);
+    io.rc = rows_of(io.row0, io.cap);
+    io.nr = prof_rows < 0 ? (double)io.cap
+                          : (double)std::max(0LL, std::min<long long>(io.cap, prof_rows - io.row0));
+    io.MT = cdiv(io.cap, PM);
+    io.row_blocks = (int)cdiv(io.cap, ROW_WARPS);
     if (list) {
-      __nv_bfloat16* hdst = hstage + (size_t)(c % G) * L.C * L.H;
-      {
-        ProfScope ps(K_GATHER, st, 0.0, nr * (L.H * 4.0 + K * 16.0 + 5.0));
-        FCKL_LAUNCH(k_gather_rows, cap, 128, 0, rowlist + row0, rc, (long long)L.N, H, K,
-                    static_cast<const __nv_bfloat16*>(q.hidden), q.topk_idx, q.topk_logit, hdst,
-                    idstage, lgstage, mstage,
-                    bwd ? reinterpret_cast<uint4*>(dlog + (size_t)(c % G) * L.C * L.Vp) : nullptr,
-                    (long long)(L.Vp / 8));
-      }
-      h_c = hdst; ids_c = idstage; lg_c = lgstage; rl_c = rlstage; dH_c = dhstage;
-      mask_c = compact ? nullptr : mstage;  // compacted rows are all valid
+      io.h = hslot(c); io.ids = idstage; io.lg = lgstage; io.rl = rlstage; io.dH = dhstage;
+      io.mask = compact ? nullptr : mstage;  // compacted rows are all valid
     } else {
-      h_c = static_cast<const uint8_t*>(q.hidden) + (size_t)row0 * L.H * 2;
-      ids_c = q.topk_idx ? q.topk_idx + row0 * K : nullptr;
-      lg_c = q.topk_logit ? q.topk_logit + row0 * K : nullptr;
-      mask_c = q.row_mask ? q.row_mask + row0 : nullptr;
-      rl_c = rl + row0;
-      dH_c = bwd ? q.dH + row0 * L.H : nullptr;
+      io.h = static_cast<const uint8_t*>(q.hidden) + (size_t)io.row0 * L.H * 2;
+      io.ids = q.topk_idx ? q.topk_idx + io.row0 * K : nullptr;
+      io.lg = q.topk_logit ? q.topk_logit + io.row0 * K : nullptr;
+      io.mask = q.row_mask ? q.row_mask + io.row0 : nullptr;
+      io.rl = rl + io.row0;
+      io.dH = bwd ? q.dH + io.row0 * L.H : nullptr;
     }
-    // This chunk's rows in the group's dlogits block.
-    __nv_bfloat16* dlog_c = dlog + (size_t)(c % G) * L.C * L.Vp;
+    io.dlog = dlog + (size_t)(c % G) * L.C * L.Vp;
+    return io;
+  };
+  // What chunk c needs before its forward GEMM: its host-input piece, its
+  // gathered rows (listed and compacted calls) and the teacher preparation
+  // (which also zeroes the chunk's dH rows for the dH GEMM's reduce-adds).
+  auto stage_in = [&](long long c, const ChunkIO& io) -> fckl_status {
+    if (q.ready && cudaStreamWaitEvent(st, q.ready[1 + c], 0) != cudaSuccess) return FCKL_ERR_CUDA;
+    if (list) {
+      // A compacted chunk zeroes the dlogits rows just past its last valid row
+      // (the dW GEMM reads whole 64-row blocks, which may reach into the next
+      // chunk's slot of the group).  The first chunk of a group leaves this to
+      // its recompute GEMM, because the previous group's dW GEMM may still be
+      // reading that slot when the gather runs.
+      uint4* dlz = (bwd && compact && c % G != 0) ? reinterpret_cast<uint4*>(io.dlog) : nullptr;
+      ProfScope ps(K_GATHER, st, 0.0, io.nr * (L.H * 4.0 + K * 16.0 + 5.0));
+      FCKL_LAUNCH(k_gather_rows, io.cap, 128, 0, rowlist + io.row0, io.rc, (long long)L.N, H, K,
+                  static_cast<const __nv_bfloat16*>(q.hidden), q.topk_idx, q.topk_logit,
+                  static_cast<__nv_bfloat16*>(const_cast<void*>(io.h)), idstage, lgstage, mstage,
+                  dlz, (long long)(L.Vp / 8));
+    }
+    if (!ent) {
+      ProfScope ps(K_PREP, st, 0.0, io.nr * K * 20.0 + io.nr * (NT + 1) * 2.0);
+      FCKL_LAUNCH(k_prep_teacher, io.row_blocks, ROW_WARPS * 32, 0, io.ids, io.lg, io.mask, io.rc,
+                  K, V, (int)NT, invT, prob->teacher == FCKL_TEACHER_PROBS, sid, sp, zs, tstart,
+                  plogp, ctl, bwd ? io.dH : (float*)nullptr, H);
+    }
+    return FCKL_OK;
+  };
 
+  ChunkIO io = chunk_io(0);
+  if (const fckl_status s0 = stage_in(0, io); s0 != FCKL_OK) return s0;
+  for (long long c = 0; c < nchunks; ++c) {
+    const bool more = c + 1 < nchunks;
     CUtensorMap mapH_k;
-    if (!make_map(&mapH_k, h_c, L.H, cap, L.H * 2, BK, CM)) return FCKL_ERR_CUDA;
+    if (!make_map(&mapH_k, io.h, L.H, io.cap, L.H * 2, BK, CM)) return FCKL_ERR_CUDA;
     // Forward units are vocab-major so that concurrent pairs share W tiles.
-    SchedArgs sa_v{SCHED_VOCAB_MAJOR, (int)NT, (int)KBh, 1, 0, rc, 0, 0};
-    const int Gv = grid_for(MT * NT);
-    const double gemm_flops = 2.0 * nr * (double)L.V * (double)L.H;
+    SchedArgs sa_v{SCHED_VOCAB_MAJOR, (int)NT, (int)KBh, 1, 0, io.rc, 0, 0};
+    const int Gv = grid_for(io.MT * NT);
+    const double gemm_flops = 2.0 * io.nr * (double)L.V * (double)L.H;
 
     if (ent) {  // student entropy: forward GEMM with the entropy epilogue, then merge
       EpiEntropy::Params pe{V, 1, (int)NT, scale2, nullptr, nullptr, nullptr, part, upart};
       {
-        ProfScope ps(K_ENT, st, gemm_flops, 2.0 * (nr + (double)L.V) * L.H + nr * NT * 12.0);
+        ProfScope ps(K_ENT, st, gemm_flops, 2.0 * (io.nr + (double)L.V) * L.H + io.nr * NT * 12.0);
         FCKL_LAUNCH((gemm_pair_kernel<EpiEntropy, false, false>), Gv, GEMM_THREADS,
                     pair_smem_bytes<EpiEntropy>(), mapH_k, mapW_k, mapW_k, pe, sa_v, ca);
       }
       {
-        ProfScope ps(K_ENT_MERGE, st, 0.0, nr * NT * 12.0 + nr * 5.0);
-        FCKL_LAUNCH(k_merge_entropy, row_blocks, ROW_WARPS * 32, 0, (const float2*)part,
-                    (const float*)upart, (int)NT, rc, mask_c, q.entropy + row0);
+        ProfScope ps(K_ENT_MERGE, st, 0.0, io.nr * NT * 12.0 + io.nr * 5.0);
+        FCKL_LAUNCH(k_merge_entropy, io.row_blocks, ROW_WARPS * 32, 0, (const float2*)part,
+                    (const float*)upart, (int)NT, io.rc, io.mask, q.entropy + io.row0);
+      }
+      if (more) {
+        io = chunk_io(c + 1);
+        if (const fckl_status s1 = stage_in(c + 1, io); s1 != FCKL_OK) return s1;
       }
       continue;
     }
 
-    {
-      ProfScope ps(K_PREP, st, 0.0, nr * K * 20.0 + nr * (NT + 1) * 2.0);
-      // prep also zeroes the chunk's dH rows, into which the dH GEMM reduce-adds
-      FCKL_LAUNCH(k_prep_teacher, row_blocks, ROW_WARPS * 32, 0, ids_c, lg_c, mask_c, rc, K, V,
-                  (int)NT, invT, prob->teacher == FCKL_TEACHER_PROBS, sid, sp, zs, tstart, plogp,
-                  ctl, bwd ? dH_c : (float*)nullptr, H);
-    }
+    // Forward: the main loop reads h and W only, complete before the kernel
+    // ahead of it launched (the gather ran before the teacher prep), so it
+    // starts at once -- possibly over the tail of the previous chunk's dW
+    // GEMM -- and only the epilogue waits.
+    SchedArgs sa_f = sa_v;
+    sa_f.early = 1;
     EpiLse::Params pf{V, K, (int)NT, scale2, sid, tstart, zs, part, nullptr};
     CtlArgs ca_f = ca;
     ca_f.debug_skip_commit = (c == 0) ? ca.debug_skip_commit : 0;
     {
-      ProfScope ps(K_FWD, st, gemm_flops, 2.0 * (nr + (double)L.V) * L.H + nr * NT * 8.0);
+      ProfScope ps(K_FWD, st, gemm_flops, 2.0 * (io.nr + (double)L.V) * L.H + io.nr * NT * 8.0);
       FCKL_LAUNCH((gemm_pair_kernel<EpiLse, false, false>), Gv, GEMM_THREADS,
-                  pair_smem_bytes<EpiLse>(), mapH_k, mapW_k, mapW_k, pf, sa_v, ca_f);
+                  pair_smem_bytes<EpiLse>(), mapH_k, mapW_k, mapW_k, pf, sa_f, ca_f);
     }
     {
-      ProfScope ps(K_MERGE, st, 0.0, nr * K * 8.0 + nr * NT * 8.0 + nr * 13.0);
-      FCKL_LAUNCH(k_merge_loss, row_blocks, ROW_WARPS * 32, 0, (const float2*)part, (int)NT, rc,
-                  K, invT, (const float*)zs, (const float*)sp, (const float*)plogp, mask_c, lse2,
-                  rl_c);
+      ProfScope ps(K_MERGE, st, 0.0, io.nr * K * 8.0 + io.nr * NT * 8.0 + io.nr * 13.0);
+      FCKL_LAUNCH(k_merge_loss, io.row_blocks, ROW_WARPS * 32, 0, (const float2*)part, (int)NT,
+                  io.rc, K, invT, (const float*)zs, (const float*)sp, (const float*)plogp, io.mask,
+                  lse2, io.rl);
     }
     if (!bwd) {
       if (list) {
-        ProfScope ps(K_SCATTER, st, 0.0, nr * 12.0);
-        FCKL_LAUNCH(k_scatter_rows, cap, 128, 0, rowlist + row0, rc, (long long)L.N, H,
+        ProfScope ps(K_SCATTER, st, 0.0, io.nr * 12.0);
+        FCKL_LAUNCH(k_scatter_rows, io.cap, 128, 0, rowlist + io.row0, io.rc, (long long)L.N, H,
                     (const float*)rlstage, rl, (const float*)nullptr, (float*)nullptr);
+      }
+      if (more) {
+        io = chunk_io(c + 1);
+        if (const fckl_status s1 = stage_in(c + 1, io); s1 != FCKL_OK) return s1;
       }
       continue;
     }
@@ -591,14 +635,16 @@ fckl_status run(const Request& q) {
     // Backward 1: recompute the tiles and form bf16 dlogits = q - p~.  Its
     // operands (h, W) were complete before the kernel ahead of it launched, so
     // its main loop starts at once and only its epilogue waits for the merge.
-    EpiDlogits::Params pb{V, K, (int)NT, scale2, lse2, sid, tstart, sp, mask_c};
+    // Rows past the chunk's last row, up to the next multiple of 64 (within
+    // the chunk), are stored as zeros for the dW GEMM's last 64-row block.
+    EpiDlogits::Params pb{V, K, (int)NT, scale2, lse2, sid, tstart, sp, io.mask, io.cap};
     SchedArgs sa_b = sa_v;
     sa_b.early = 1;
     CUtensorMap mapD_st;
     // The store map spans the padded width: the pad columns receive zeros.
-    if (!make_map(&mapD_st, dlog_c, L.Vp, cap, L.Vp * 2, 64, 32)) return FCKL_ERR_CUDA;
+    if (!make_map(&mapD_st, io.dlog, L.Vp, io.cap, L.Vp * 2, 64, 32)) return FCKL_ERR_CUDA;
     {
-      ProfScope ps(K_BWD, st, gemm_flops, 2.0 * (nr + (double)L.V) * L.H + 2.0 * nr * L.V);
+      ProfScope ps(K_BWD, st, gemm_flops, 2.0 * (io.nr + (double)L.V) * L.H + 2.0 * io.nr * L.V);
       FCKL_LAUNCH((gemm_pair_kernel<EpiDlogits, false, false>), Gv, GEMM_THREADS,
                   pair_smem_bytes<EpiDlogits>(), mapH_k, mapW_k, mapD_st, pb, sa_b, ca);
     }
@@ -606,36 +652,43 @@ fckl_status run(const Request& q) {
     // Backward 2: dH[rows] = alpha * dlogits W; A = dlogits (K-major), B = W (MN-major),
     // reduce-added into the rows k_prep_teacher zeroed.
     CUtensorMap mapD_k, mapD_mn, mapH_mn, mapdH;
-    if (!make_map(&mapD_k, dlog_c, L.V, cap, L.Vp * 2, BK, CM)) return FCKL_ERR_CUDA;
-    if (!make_map(&mapdH, dH_c, L.H, cap, L.H * 4, 32, 32, true)) return FCKL_ERR_CUDA;
-    const long long tiles_h = MT * NTh;
+    if (!make_map(&mapD_k, io.dlog, L.V, io.cap, L.Vp * 2, BK, CM)) return FCKL_ERR_CUDA;
+    if (!make_map(&mapdH, io.dH, L.H, io.cap, L.H * 4, 32, 32, true)) return FCKL_ERR_CUDA;
+    const long long tiles_h = io.MT * NTh;
     // A compacted chunk's row count is only known on the device: the kernel
     // picks the split there (S = 0) and the launch covers every pair.
     const int S = compact ? 0 : choose_split(tiles_h, KBv, pairs);
-    SchedArgs sa_h{SCHED_SPLIT_K, (int)NTh, (int)KBv, S, 0, rc, 0, w3d, 0, narrow_h, 0,
+    SchedArgs sa_h{SCHED_SPLIT_K, (int)NTh, (int)KBv, S, 0, io.rc, 0, w3d, 0, narrow_h, 0,
                    dh_tile_order(), dh_serpentine()};
     EpiDH::Params ph{H, invT, ctl};
     {
       ProfScope ps(K_DH, st, gemm_flops,
-                   2.0 * nr * (double)L.V + 2.0 * (double)L.V * L.H + 4.0 * nr * L.H);
+                   2.0 * io.nr * (double)L.V + 2.0 * (double)L.V * L.H + 4.0 * io.nr * L.H);
       FCKL_LAUNCH((gemm_pair_kernel<EpiDH, false, true>),
                   S > 0 ? grid_for(tiles_h * S) : 2 * pairs, GEMM_THREADS, pair_smem_bytes<EpiDH>(),
                   mapD_k, mapW_mn, mapdH, ph, sa_h, ca);
     }
     if (list) {
-      ProfScope ps(K_SCATTER, st, 0.0, nr * (12.0 + 8.0 * L.H));
-      FCKL_LAUNCH(k_scatter_rows, cap, 128, 0, rowlist + row0, rc, (long long)L.N, H,
+      ProfScope ps(K_SCATTER, st, 0.0, io.nr * (12.0 + 8.0 * L.H));
+      FCKL_LAUNCH(k_scatter_rows, io.cap, 128, 0, rowlist + io.row0, io.rc, (long long)L.N, H,
                   (const float*)rlstage, rl, (const float*)dhstage, q.dH);
+    }
+    const ChunkIO cur = io;
+    // The next chunk's gather and teacher prep go ahead of this group's dW
+    // GEMM, so that the next forward GEMM can follow the dW GEMM directly.
+    if (more) {
+      io = chunk_io(c + 1);
+      if (const fckl_status s1 = stage_in(c + 1, io); s1 != FCKL_OK) return s1;
     }
 
     // Backward 3, once per group of G chunks (or at the last chunk):
     // dW (+)= alpha * dlogits^T h over the group's rows; A = dlogits^T, B = h
     // (both MN-major).
-    if ((c + 1) % G != 0 && c + 1 != nchunks) continue;
+    if ((c + 1) % G != 0 && more) continue;
     const long long g0 = c / G * G;  // first chunk of the group
     const long long grow0 = g0 * L.C;
-    const int gcap = (int)(row0 + cap - grow0);
-    const void* h_g = list ? static_cast<const void*>(hstage)
+    const int gcap = (int)(cur.row0 + cur.cap - grow0);
+    const void* h_g = list ? static_cast<const void*>(hslot(g0))
                            : static_cast<const uint8_t*>(q.hidden) + (size_t)grow0 * L.H * 2;
     int d3d = 0, h3d = 0;
     if (!make_map_mn(&mapD_mn, dlog, L.Vp, gcap, L.Vp * 2, &d3d)) return FCKL_ERR_CUDA;
@@ -649,7 +702,7 @@ fckl_status run(const Request& q) {
     }
     // One launch over all vocabulary tiles, or -- for the last group of a
     // sliced call -- one launch per slice, each followed by its event.
-    const bool sliced = q.n_slices > 0 && c + 1 == nchunks;
+    const bool sliced = q.n_slices > 0 && !more;
     const long long ns = sliced ? std::min<long long>(q.n_slices, MTv) : 1;
     const double gr = prof_rows < 0
                           ? (double)gcap

@@ -90,7 +90,12 @@ def test_workspace_follows_an_explicit_chunk():
     N, H, V, K = 131072, 2880, 201088, 100
     Vp = (V + 63) // 64 * 64
     small = fk.fckl_workspace_bytes(FcklProblem(N, H, V, K, 1.0, 256))
-    assert 256 * Vp * 2 + N * 8 <= small < 256 * Vp * 2 + N * 8 + 8 * 2**20
+    # per-chunk buffers: 14 bytes per row and vocab tile of 256 (partials,
+    # tile starts), 12 per hidden unit (two staged hidden rows, one fp32 dH
+    # row), about 36 per teacher entry
+    NT = (V + 255) // 256
+    per_chunk = 256 * (14 * NT + 12 * H + 36 * K + 64)
+    assert 256 * Vp * 2 + N * 8 <= small < 256 * Vp * 2 + N * 8 + per_chunk + 2**20
     big = fk.fckl_workspace_bytes(FcklProblem(N, H, V, K, 1.0, 2048))
     assert big - small >= (2048 - 256) * Vp * 2
     # linear in the chunk beyond the per-row arrays

@@ -74,10 +74,11 @@ def _check_rows(inp, rows_np, T, chunk):
     # the same as the masked full-row call
     l2, _, dH2, dW2 = fused_kl_fwd_bwd(d[0], d[1], d[2], d[3], torch.from_numpy(mask).cuda(), T=T,
                                        chunk=chunk)
-    # dH sums V terms in fp32 split-K segments whose count can differ between
-    # the two calls (a host row count vs a device one): reassociation only
+    # dH's split-K partial sums reach dH through fp32 reduce-adds in whatever
+    # order the units finish; both calls pick the same split from the same row
+    # count, so the two differ by that reassociation only (measured <= 1.3e-7)
     assert abs(l2.item() - loss.item()) <= 1e-5 * abs(loss.item())
-    assert rel_fro(dH.cpu().numpy(), dH2.cpu().numpy()) < 5e-4
+    assert rel_fro(dH.cpu().numpy(), dH2.cpu().numpy()) < 1e-5
     assert rel_fro(dW.cpu().numpy(), dW2.cpu().numpy()) < 1e-5
 
 
