@@ -88,6 +88,8 @@ def parse():
                     help="print peak device memory vs sequence length instead of timing")
     ap.add_argument("--sweep-chunk", type=int, default=2048,
                     help="--mem-sweep: rows per chunk")
+    ap.add_argument("--sweep-s", default="8192,16384,32768,65536,131072,262144",
+                    help="--mem-sweep: comma-separated sequence lengths")
     ap.add_argument("--vs-cublas", type=float, default=0.0, metavar="SECONDS",
                     help="instead of the contract line: run the fused step and the four plain "
                          "cuBLAS GEMMs of the same shapes back to back for SECONDS each, clocks "
@@ -245,14 +247,22 @@ def run_cuda(args):
     rank, local, world = dist_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    mode = "single" if world == 1 else (args.mode or "dp")
-    if world > 1:
+    # one GPU: the plain fused call, unless --mode dp asks for the data-parallel
+    # path on a one-rank process group (its collectives then run on one rank)
+    mode = (args.mode if args.mode == "dp" else "single") if world == 1 else (args.mode or "dp")
+    use_pg = world > 1 or mode == "dp"
+    if use_pg:
         import datetime
+        if "MASTER_ADDR" not in os.environ:
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            os.environ.setdefault("MASTER_PORT", "29511")
+            os.environ.setdefault("RANK", "0")
+            os.environ.setdefault("WORLD_SIZE", "1")
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
 
     def barrier():
-        if world > 1:
+        if use_pg:
             dist.barrier()
 
     cfg = workload(args)
@@ -403,7 +413,7 @@ def run_cuda(args):
         if args.profile_json:
             with open(args.profile_json, "w") as fh:
                 json.dump(line, fh, indent=1)
-    if world > 1:
+    if use_pg:
         dist.barrier()
         dist.destroy_process_group()
     return 0
@@ -535,7 +545,7 @@ def run_mem_sweep(args):
     torch.cuda.set_device(0)
     H, V, K, C = 4096, 128256, 100, args.sweep_chunk
     pts = []
-    for S in (8192, 16384, 32768, 65536, 131072, 262144):
+    for S in [int(x) for x in args.sweep_s.split(",") if x]:
         torch.cuda.empty_cache()
         base = torch.cuda.memory_allocated()
         g = torch.Generator(device="cuda").manual_seed(S)

@@ -15,12 +15,15 @@ constexpr uint32_t kErrBadTeacher = 2u;
 constexpr uint32_t kErrTimeout = 4u;
 
 // First 256 bytes of every workspace.
+constexpr int kCompactBlocks = 48;  // blocks of the two-pass valid-row compaction
+
 struct DeviceCtl {
   uint32_t err;       // OR of kErr* bits
   int32_t n_valid;    // number of rows with row_mask != 0
   uint32_t timeout_site;  // which wait gave up first (diagnostics)
   int32_t n_rows;     // rows a masked call compacted (its local valid rows)
-  uint32_t pad[60];
+  int32_t block_count[kCompactBlocks];  // valid rows per compaction block
+  uint32_t pad[60 - kCompactBlocks];
 };
 static_assert(sizeof(DeviceCtl) == 256, "control block is 256 bytes");
 

@@ -23,6 +23,11 @@ __device__ __forceinline__ float warp_sum(float x) {
   for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
   return x;
 }
+__device__ __forceinline__ int warp_sum_int(int x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
 
 // N_valid = #rows with row_mask != 0 (N when there is no mask), or the
 // caller's total (> 0) when the rows are one shard of a larger batch.  One block.
@@ -75,14 +80,6 @@ __global__ void __launch_bounds__(1024) k_count_list(const int32_t* __restrict__
     if (threadIdx.x == 0) ctl->n_valid = total > 0 ? total : c;
   }
 }
-
-// Row indices of the valid rows (row_mask != 0), ascending, into list[0, n),
-// n into ctl->n_rows and N_v (n, or the caller's global total when > 0) into
-// ctl->n_valid.  One block: each thread scans a contiguous range; a block-wide
-// prefix sum gives every thread its output position.
-__global__ void __launch_bounds__(1024) k_compact_mask(const uint8_t* __restrict__ mask,
-                                                       long long N, int total,
-                                                       int32_t* __restrict__ list, DeviceCtl* ctl);
 
 // dW = 0 when the call compacted no row (then no dW launch writes it);
 // otherwise nothing.
@@ -186,23 +183,68 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* sh, int* total) 
   return before;
 }
 
-__global__ void __launch_bounds__(1024) k_compact_mask(const uint8_t* __restrict__ mask,
-                                                       long long N, int total,
-                                                       int32_t* __restrict__ list, DeviceCtl* ctl) {
+// Row indices of the valid rows (row_mask != 0), ascending, into list[0, n),
+// n into ctl->n_rows and N_v (n, or the caller's global total when > 0) into
+// ctl->n_valid, in two passes over kCompactBlocks blocks: block b owns rows
+// [b*R, (b+1)*R) (R a multiple of 4096).  Pass 1 counts each block's valid
+// rows into ctl->block_count[b]; pass 2 starts block b at the sum of the
+// counts before it and writes its rows 4096 at a time (thread t takes 4
+// consecutive rows; a block-wide prefix sum gives every thread its position).
+__global__ void __launch_bounds__(1024) k_compact_count(const uint8_t* __restrict__ mask,
+                                                        long long N, long long R, DeviceCtl* ctl) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ int red[32];
+  const long long r0 = blockIdx.x * R, r1 = (r0 + R < N) ? r0 + R : N;
+  int c = 0;
+  for (long long i = r0 + threadIdx.x; i < r1; i += blockDim.x) c += mask[i] != 0;
+  c = warp_sum_int(c);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = c;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    c = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0;
+    c = warp_sum_int(c);
+    if (threadIdx.x == 0) ctl->block_count[blockIdx.x] = c;
+  }
+}
+
+__global__ void __launch_bounds__(1024) k_compact_write(const uint8_t* __restrict__ mask,
+                                                        long long N, long long R, int total,
+                                                        int32_t* __restrict__ list,
+                                                        DeviceCtl* ctl) {
   pdl_wait();
   pdl_trigger();
   __shared__ int sh[32];
-  const long long per = (N + blockDim.x - 1) / blockDim.x;
-  const long long i0 = threadIdx.x * per, i1 = (i0 + per < N) ? i0 + per : N;
-  int cnt = 0;
-  for (long long i = i0; i < i1; ++i) cnt += mask[i] != 0;
-  int count;
-  int pos = block_exclusive_scan(cnt, sh, &count);
-  for (long long i = i0; i < i1; ++i)
-    if (mask[i] != 0) list[pos++] = (int32_t)i;
+  __shared__ int s_base, s_total;
   if (threadIdx.x == 0) {
-    ctl->n_rows = count;
-    ctl->n_valid = total > 0 ? total : count;
+    int before = 0, all = 0;
+    for (int b = 0; b < (int)gridDim.x; ++b) {
+      const int cb = ctl->block_count[b];
+      before += b < (int)blockIdx.x ? cb : 0;
+      all += cb;
+    }
+    s_base = before;
+    s_total = all;
+  }
+  __syncthreads();
+  int base = s_base;
+  const long long r0 = blockIdx.x * R, r1 = (r0 + R < N) ? r0 + R : N;
+  for (long long t0 = r0; t0 < r1; t0 += 4 * (long long)blockDim.x) {
+    const long long i0 = t0 + 4 * (long long)threadIdx.x;
+    int f = 0;  // bit k: row i0 + k is valid
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (i0 + k < r1 && mask[i0 + k] != 0) f |= 1 << k;
+    int tile_total;
+    int pos = base + block_exclusive_scan(__popc(f), sh, &tile_total);
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (f & (1 << k)) list[pos++] = (int32_t)(i0 + k);
+    base += tile_total;
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    ctl->n_rows = s_total;
+    ctl->n_valid = total > 0 ? total : s_total;
   }
 }
 

@@ -94,7 +94,9 @@ typedef enum {
  * "chunked KL loss가 하는 일").  dw_rows > chunk groups ceil(dw_rows / chunk)
  * consecutive chunks into one dW GEMM (at most all of them): fewer
  * read-modify-writes of the fp32 dW (V * H * 8 bytes each) for small chunks,
- * at the price of a workspace holding the whole group's dlogits. */
+ * at the price of a workspace holding the whole group's dlogits.  With
+ * chunk = 0 and dw_rows = 0 the library also picks the grouping: at least
+ * 4096 rows per dW GEMM (e.g. two automatic 2560-row chunks at V = 201,088). */
 typedef struct {
   int64_t N;        /* rows (batch * sequence)                  */
   int64_t H;        /* hidden size                              */
@@ -107,9 +109,10 @@ typedef struct {
                             > 0: N_v used for the mean and the gradient
                             scale, e.g. the valid rows of all data-parallel
                             ranks, each rank passing its own row shard */
-  int64_t dw_rows;  /* 0: one dW GEMM per chunk; > 0: each dW GEMM
-                       reduces over at least this many rows (chunks
-                       grouped; see above).  0 <= dw_rows <= INT32_MAX */
+  int64_t dw_rows;  /* 0: one dW GEMM per chunk (automatic chunk: at
+                       least 4096 rows); > 0: each dW GEMM reduces over at
+                       least this many rows (chunks grouped; see above).
+                       0 <= dw_rows <= INT32_MAX */
 } fckl_problem;
 
 /* What the teacher cache holds in topk_logit [N, K]:

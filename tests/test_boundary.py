@@ -62,6 +62,15 @@ def test_workspace_and_chunk_rules():
     assert b - a == 32768 * 8    # only the per-row loss and the compacted row list grow
     # an explicit chunk bounds the dlogits block: one chunk of bf16 dlogits
     assert 1024 * 128256 * 2 <= a < 1024 * 128256 * 2 + 48 * 2**20
+    # the automatic chunk also picks the grouping (>= 4096 rows per dW GEMM):
+    # two 2560-row chunks at the gpt-oss vocabulary; the same explicit chunk
+    # keeps one chunk of dlogits
+    Vp3 = (201088 + 63) // 64 * 64
+    auto3 = fk.fckl_workspace_bytes(p3)
+    expl3 = fk.fckl_workspace_bytes(FcklProblem(131072, 2880, 201088, 100, 1.0, 2560))
+    assert auto3 - expl3 >= 2560 * Vp3 * 2 and expl3 < 2 * 2560 * Vp3 * 2
+    assert fk.fckl_workspace_bytes(FcklProblem(131072, 2880, 201088, 100, 1.0, 0,
+                                               dw_rows=1)) == expl3
     # dw_rows = 4096 groups four 1024-row chunks into one dW GEMM
     g = fk.fckl_workspace_bytes(FcklProblem(32768, 4096, 128256, 100, 1.0, 1024, dw_rows=4096))
     assert g - a >= 3 * 1024 * 128256 * 2 + 3 * 1024 * 4096 * 2
