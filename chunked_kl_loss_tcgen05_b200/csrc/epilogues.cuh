@@ -12,7 +12,8 @@
 //               rounded once to bf16, staged in shared memory and
 //               TMA-stored to the chunk's dlogits block.
 //   EpiDH       dH[rows, :] += alpha * (dlogits W) partial (split-K): fp32
-//               tile staged in shared memory, TMA reduce-add into dH.
+//               tile staged in shared memory, TMA reduce-add into dH (or,
+//               for gathered rows, vector reductions into the caller's rows).
 //   EpiDW       dW (+)= alpha * (dlogits^T h): TMA store (first chunk) or
 //               TMA reduce-add (later chunks), so the fp32 read-modify-write
 //               of dW happens in L2, coalesced and off the epilogue threads.
@@ -272,6 +273,28 @@ __device__ __forceinline__ void stage_fp32_slices(uint8_t* bufs, int& n, uint32_
   }
 }
 
+// dH of gathered rows goes straight to the caller's dH rows: the staged slice
+// is read back 4 rows x 128 bytes per warp instruction and added with vector
+// reductions at dH + out_rows[row] * H (rows outside [0, N) are skipped).
+__device__ __forceinline__ void reduce_slice_to_rows(const uint8_t* buf, int lane, int y_local,
+                                                     int rows, const int32_t* out_rows,
+                                                     long long N, float* out, int H, int x) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int rr = i * 4 + (lane >> 3), ch = lane & 7;
+    const int row = y_local + rr;
+    if (row >= rows || x + ch * 4 >= H) continue;
+    const int r = __ldg(out_rows + row);
+    if (r < 0 || r >= N) continue;
+    const uint4 q = *reinterpret_cast<const uint4*>(buf + rr * 128 + ((ch ^ (rr & 7)) << 4));
+    float* dst = out + (size_t)r * H + x + ch * 4;
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst),
+                 "f"(__uint_as_float(q.x)), "f"(__uint_as_float(q.y)), "f"(__uint_as_float(q.z)),
+                 "f"(__uint_as_float(q.w))
+                 : "memory");
+  }
+}
+
 struct EpiDH {
   static constexpr uint32_t kSmemBytes = 4 * 2 * 4096;
   static constexpr bool kUsesMapC = true;  // map C: dH chunk rows [rows, H] fp32, box {32, 32}
@@ -279,6 +302,12 @@ struct EpiDH {
     int H;
     float invT;
     const DeviceCtl* ctl;
+    // Gathered rows: the caller's row of each chunk row (nullptr: the chunk's
+    // rows are contiguous rows of dH and map C covers them), the caller's dH
+    // and its row count.
+    const int32_t* out_rows;
+    float* out;
+    long long N;
   };
   struct State {
     float alpha;
@@ -294,7 +323,25 @@ struct EpiDH {
   static __device__ void tile(const Params& p, State& st, const Work& w, uint32_t taddr, int,
                               const CUtensorMap* mapC, int quarter, int lane) {
     const int y = w.m0 + quarter * 32;
-    stage_fp32_slices<true>(st.buf, st.n, taddr, st.alpha, mapC, w.n0, p.H, y, y < w.rows, lane);
+    if (p.out_rows == nullptr) {
+      stage_fp32_slices<true>(st.buf, st.n, taddr, st.alpha, mapC, w.n0, p.H, y, y < w.rows, lane);
+      return;
+    }
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      float v[32];
+      tmem_ld32_conv(taddr + (uint32_t)(c * 32), v);
+      if (y >= w.rows) continue;
+      uint8_t* buf = st.buf;
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        *stage_chunk(buf, lane, j) =
+            make_uint4(__float_as_uint(st.alpha * v[4 * j]), __float_as_uint(st.alpha * v[4 * j + 1]),
+                       __float_as_uint(st.alpha * v[4 * j + 2]), __float_as_uint(st.alpha * v[4 * j + 3]));
+      __syncwarp();
+      reduce_slice_to_rows(buf, lane, y, w.rows, p.out_rows, p.N, p.out, p.H, w.n0 + c * 32);
+      __syncwarp();
+    }
   }
   static __device__ void finish(const Params&, State&, int lane) {
     if (lane == 0) bulk_wait_all();

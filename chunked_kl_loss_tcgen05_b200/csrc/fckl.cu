@@ -37,8 +37,7 @@ struct Layout {
   long long N, H, V, K, C, Vp, nchunks, NT;
   long long G;  // chunks per dW group: dlogits of G chunks feed one dW GEMM
   size_t off_rowloss, off_sid, off_sp, off_zs, off_tstart, off_plogp, off_lse2, off_part,
-      off_upart, off_hstage, off_idstage, off_lgstage, off_mstage, off_dhstage, off_rlstage,
-      off_list, off_dlog, total;
+      off_upart, off_hstage, off_idstage, off_lgstage, off_mstage, off_list, off_dlog, total;
 };
 
 bool valid_problem(const fckl_problem* p) {
@@ -108,8 +107,6 @@ Layout make_layout(const fckl_problem* p, bool full = true) {
   L.off_idstage = take(full ? C * L.K * 4 : 0);
   L.off_lgstage = take(full ? C * L.K * 4 : 0);
   L.off_mstage = take(full ? C : 0);
-  L.off_dhstage = take(full ? C * L.H * 4 : 0);
-  L.off_rlstage = take(full ? C * 4 : 0);
   L.off_list = take(full ? (size_t)L.N * 4 : 0);  // valid rows of a masked call, compacted
   L.off_dlog = take(full ? (size_t)L.G * C * L.Vp * 2 : 0);
   L.total = off;
@@ -426,8 +423,6 @@ fckl_status run(const Request& q) {
   int32_t* idstage = reinterpret_cast<int32_t*>(ws + L.off_idstage);
   float* lgstage = reinterpret_cast<float*>(ws + L.off_lgstage);
   uint8_t* mstage = ws + L.off_mstage;
-  float* dhstage = reinterpret_cast<float*>(ws + L.off_dhstage);
-  float* rlstage = reinterpret_cast<float*>(ws + L.off_rlstage);
   int32_t* clist = reinterpret_cast<int32_t*>(ws + L.off_list);
   __nv_bfloat16* dlog = reinterpret_cast<__nv_bfloat16*>(ws + L.off_dlog);
   const int32_t* rowlist = user_list ? q.rows : clist;
@@ -524,9 +519,10 @@ fckl_status run(const Request& q) {
     const int32_t* ids;
     const float* lg;
     const uint8_t* mask;
-    float* rl;
-    float* dH;
-    __nv_bfloat16* dlog;  // this chunk's rows in the group's dlogits block
+    float* rl;               // row loss of the chunk's first row (out_rows == nullptr)
+    float* dH;               // dH of the chunk's first row (out_rows == nullptr)
+    const int32_t* out_rows; // gathered rows: the caller's row of each chunk row
+    __nv_bfloat16* dlog;     // this chunk's rows in the group's dlogits block
   };
   auto hslot = [&](long long c) {
     return hstage + (size_t)(((c / G) & 1) * G + c % G) * L.C * L.H;
@@ -541,9 +537,13 @@ fckl_status run(const Request& q) {
     io.MT = cdiv(io.cap, PM);
     io.row_blocks = (int)cdiv(io.cap, ROW_WARPS);
     if (list) {
-      io.h = hslot(c); io.ids = idstage; io.lg = lgstage; io.rl = rlstage; io.dH = dhstage;
+      // row losses and dH rows go straight to the caller's rows (dH was zeroed
+      // at the start of the call)
+      io.h = hslot(c); io.ids = idstage; io.lg = lgstage; io.rl = rl; io.dH = nullptr;
+      io.out_rows = rowlist + io.row0;
       io.mask = compact ? nullptr : mstage;  // compacted rows are all valid
     } else {
+      io.out_rows = nullptr;
       io.h = static_cast<const uint8_t*>(q.hidden) + (size_t)io.row0 * L.H * 2;
       io.ids = q.topk_idx ? q.topk_idx + io.row0 * K : nullptr;
       io.lg = q.topk_logit ? q.topk_logit + io.row0 * K : nullptr;
@@ -576,7 +576,7 @@ fckl_status run(const Request& q) {
       ProfScope ps(K_PREP, st, 0.0, io.nr * K * 20.0 + io.nr * (NT + 1) * 2.0);
       FCKL_LAUNCH(k_prep_teacher, io.row_blocks, ROW_WARPS * 32, 0, io.ids, io.lg, io.mask, io.rc,
                   K, V, (int)NT, invT, prob->teacher == FCKL_TEACHER_PROBS, sid, sp, zs, tstart,
-                  plogp, ctl, bwd ? io.dH : (float*)nullptr, H);
+                  plogp, ctl, io.dH, H);
     }
     return FCKL_OK;
   };
@@ -629,14 +629,9 @@ fckl_status run(const Request& q) {
       ProfScope ps(K_MERGE, st, 0.0, io.nr * K * 8.0 + io.nr * NT * 8.0 + io.nr * 13.0);
       FCKL_LAUNCH(k_merge_loss, io.row_blocks, ROW_WARPS * 32, 0, (const float2*)part, (int)NT,
                   io.rc, K, invT, (const float*)zs, (const float*)sp, (const float*)plogp, io.mask,
-                  lse2, io.rl);
+                  lse2, io.rl, io.out_rows, (long long)L.N);
     }
     if (!bwd) {
-      if (list) {
-        ProfScope ps(K_SCATTER, st, 0.0, io.nr * 12.0);
-        FCKL_LAUNCH(k_scatter_rows, io.cap, 128, 0, rowlist + io.row0, io.rc, (long long)L.N, H,
-                    (const float*)rlstage, rl, (const float*)nullptr, (float*)nullptr);
-      }
       if (more) {
         io = chunk_io(c + 1);
         if (const fckl_status s1 = stage_in(c + 1, io); s1 != FCKL_OK) return s1;
@@ -665,25 +660,24 @@ fckl_status run(const Request& q) {
     // reduce-added into the rows k_prep_teacher zeroed.
     CUtensorMap mapD_k, mapD_mn, mapH_mn, mapdH;
     if (!make_map(&mapD_k, io.dlog, L.V, io.cap, L.Vp * 2, BK, CM)) return FCKL_ERR_CUDA;
-    if (!make_map(&mapdH, io.dH, L.H, io.cap, L.H * 4, 32, 32, true)) return FCKL_ERR_CUDA;
+    // (gathered rows are added to the caller's rows without a map; the map
+    // then spans all of dH and is not used)
+    if (io.out_rows ? !make_map(&mapdH, q.dH, L.H, L.N, L.H * 4, 32, 32, true)
+                    : !make_map(&mapdH, io.dH, L.H, io.cap, L.H * 4, 32, 32, true))
+      return FCKL_ERR_CUDA;
     const long long tiles_h = io.MT * NTh;
     // A compacted chunk's row count is only known on the device: the kernel
     // picks the split there (S = 0) and the launch covers every pair.
     const int S = compact ? 0 : choose_split(tiles_h, KBv, pairs);
     SchedArgs sa_h{SCHED_SPLIT_K, (int)NTh, (int)KBv, S, 0, io.rc, 0, w3d, 0, narrow_h, 0,
                    dh_tile_order(), dh_serpentine()};
-    EpiDH::Params ph{H, invT, ctl};
+    EpiDH::Params ph{H, invT, ctl, io.out_rows, q.dH, (long long)L.N};
     {
       ProfScope ps(K_DH, st, gemm_flops,
                    2.0 * io.nr * (double)L.V + 2.0 * (double)L.V * L.H + 4.0 * io.nr * L.H);
       FCKL_LAUNCH((gemm_pair_kernel<EpiDH, false, true>),
                   S > 0 ? grid_for(tiles_h * S) : 2 * pairs, GEMM_THREADS, pair_smem_bytes<EpiDH>(),
                   mapD_k, mapW_mn, mapdH, ph, sa_h, ca);
-    }
-    if (list) {
-      ProfScope ps(K_SCATTER, st, 0.0, io.nr * (12.0 + 8.0 * L.H));
-      FCKL_LAUNCH(k_scatter_rows, io.cap, 128, 0, rowlist + io.row0, io.rc, (long long)L.N, H,
-                  (const float*)rlstage, rl, (const float*)dhstage, q.dH);
     }
     const ChunkIO cur = io;
     // The next chunk's gather and teacher prep go ahead of this group's dW

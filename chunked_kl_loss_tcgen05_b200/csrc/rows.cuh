@@ -131,25 +131,6 @@ __global__ void __launch_bounds__(128)
   if (threadIdx.x == 0) mst[i] = ok ? 1 : 0;
 }
 
-// Scatter one chunk's per-entry results back to the listed rows: row loss and
-// (when dH is given) the fp32 dH row.
-__global__ void __launch_bounds__(128)
-    k_scatter_rows(const int32_t* __restrict__ list, RowCount rc, long long N, int H,
-                   const float* __restrict__ rl_stage, float* __restrict__ rl,
-                   const float* __restrict__ dh_stage, float* __restrict__ dH) {
-  pdl_trigger();  // the dW GEMM after it may start its main loop
-  pdl_wait();
-  const int i = blockIdx.x;
-  if (i >= rc.get()) return;
-  const int r = list[i];
-  if (r < 0 || r >= N) return;
-  if (threadIdx.x == 0) rl[r] = rl_stage[i];
-  if (dH == nullptr) return;
-  const float4* src = reinterpret_cast<const float4*>(dh_stage + (size_t)i * H);
-  float4* dst = reinterpret_cast<float4*>(dH + (size_t)r * H);
-  for (int j = threadIdx.x; j < H / 4; j += blockDim.x) dst[j] = src[j];
-}
-
 // Order-preserving map of a float to uint32 (larger float -> larger key).
 __device__ __forceinline__ uint32_t float_key(float f) {
   const uint32_t b = __float_as_uint(f);
@@ -453,11 +434,14 @@ __global__ void __launch_bounds__(ROW_WARPS * 32)
 // Merge the per-vocab-tile (max, sum) partials of each row into its
 // log-sum-exp (log2 domain, kept for the backward epilogue) and form the row
 // loss  l_r = sum_k p_k log p_k - sum_k p_k (z_k / T - LSE_r),  0 for masked rows.
+// The row loss goes to row_loss[row], or -- for gathered rows -- to
+// row_loss[out_rows[row]] (entries outside [0, N) are skipped).
 __global__ void __launch_bounds__(ROW_WARPS * 32)
     k_merge_loss(const float2* __restrict__ partials, int NT, RowCount rc, int K, float invT,
                  const float* __restrict__ zs, const float* __restrict__ sp,
                  const float* __restrict__ plogp, const uint8_t* __restrict__ mask,
-                 float* __restrict__ lse2_out, float* __restrict__ row_loss) {
+                 float* __restrict__ lse2_out, float* __restrict__ row_loss,
+                 const int32_t* __restrict__ out_rows, long long N) {
   pdl_trigger();  // the recompute GEMM after it may start its main loop
   pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -484,7 +468,13 @@ __global__ void __launch_bounds__(ROW_WARPS * 32)
   if (lane == 0) {
     const bool keep = mask == nullptr || mask[row] != 0;
     lse2_out[row] = L2;
-    row_loss[row] = keep ? plogp[row] - acc : 0.f;
+    const float l = keep ? plogp[row] - acc : 0.f;
+    if (out_rows == nullptr) {
+      row_loss[row] = l;
+    } else {
+      const int r = out_rows[row];
+      if (r >= 0 && r < N) row_loss[r] = l;
+    }
   }
 }
 

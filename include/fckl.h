@@ -313,8 +313,9 @@ const char* fckl_status_string(fckl_status status);
  * once per call while recording is on.
  * Kinds: 0 count_valid, 1 prep_teacher, 2 fwd_logits_lse, 3 merge_loss,
  *        4 bwd_dlogits, 5 dH_gemm, 6 dW_gemm, 7 finalize, 8 entropy_gemm,
- *        9 merge_entropy, 10 gather_rows, 11 scatter_rows, 12 select_rows,
- *        13 zero_dw. */
+ *        9 merge_entropy, 10 gather_rows, 11 scatter_rows (reserved: gathered
+ *        rows write their results in place, no kernel of this kind runs),
+ *        12 select_rows, 13 zero_dw. */
 typedef struct {
   char name[32];     /* kernel kind, e.g. "fwd_logits_lse" */
   int64_t launches;  /* launches recorded */
