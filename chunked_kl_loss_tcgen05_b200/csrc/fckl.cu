@@ -370,6 +370,23 @@ struct Request {
   int64_t* slice_rows = nullptr;
 };
 
+// Per device: the library's second stream, on which the next chunk's gather
+// and teacher prep run while the current chunk's dH GEMM runs on the caller's
+// stream, and a pool of events for the hand-overs (created on first use, kept
+// until the process exits).  Calls that use it are serialised while they
+// enqueue.  FCKL_ONE_STREAM=1 keeps everything on the caller's stream.
+struct RowStream {
+  std::mutex mu;
+  cudaStream_t rs = nullptr;
+  std::vector<cudaEvent_t> ev;
+};
+RowStream g_rs[kMaxDevices];
+
+bool two_streams_enabled() {
+  const char* s = std::getenv("FCKL_ONE_STREAM");
+  return !(s && std::atoi(s) > 0);
+}
+
 fckl_status run(const Request& q) {
   const fckl_problem* prob = q.prob;
   const bool bwd = q.mode == Mode::kFwdBwd;
@@ -557,7 +574,8 @@ fckl_status run(const Request& q) {
   // What chunk c needs before its forward GEMM: its host-input piece, its
   // gathered rows (listed and compacted calls) and the teacher preparation
   // (which also zeroes the chunk's dH rows for the dH GEMM's reduce-adds).
-  auto stage_in = [&](long long c, const ChunkIO& io) -> fckl_status {
+  auto stage_in = [&](long long c, const ChunkIO& io, cudaStream_t ss) -> fckl_status {
+    cudaStream_t st = ss;  // the launches below go to this stream
     if (q.ready && cudaStreamWaitEvent(st, q.ready[1 + c], 0) != cudaSuccess) return FCKL_ERR_CUDA;
     if (list) {
       // A compacted chunk zeroes the dlogits rows just past its last valid row
@@ -581,8 +599,32 @@ fckl_status run(const Request& q) {
     return FCKL_OK;
   };
 
+  // Backward calls of several chunks run the next chunk's gather and teacher
+  // prep on the library's second stream, between the recompute GEMM and the
+  // dW GEMM of the current chunk: the teacher buffers are free once the
+  // recompute GEMM is done, and the gathered rows go to the other buffer.
+  std::unique_lock<std::mutex> rs_lock;
+  RowStream* rsd = nullptr;
+  if (bwd && nchunks > 1 && two_streams_enabled()) {
+    int dev_id = 0;
+    if (cudaGetDevice(&dev_id) != cudaSuccess || dev_id < 0 || dev_id >= kMaxDevices)
+      return FCKL_ERR_CUDA;
+    rsd = &g_rs[dev_id];
+    rs_lock = std::unique_lock<std::mutex>(rsd->mu);
+    if (rsd->rs == nullptr &&
+        cudaStreamCreateWithFlags(&rsd->rs, cudaStreamNonBlocking) != cudaSuccess) {
+      rsd->rs = nullptr;
+      return FCKL_ERR_CUDA;
+    }
+    while ((long long)rsd->ev.size() < 2 * nchunks) {
+      cudaEvent_t e = nullptr;
+      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return FCKL_ERR_CUDA;
+      rsd->ev.push_back(e);
+    }
+  }
+
   ChunkIO io = chunk_io(0);
-  if (const fckl_status s0 = stage_in(0, io); s0 != FCKL_OK) return s0;
+  if (const fckl_status s0 = stage_in(0, io, st); s0 != FCKL_OK) return s0;
   for (long long c = 0; c < nchunks; ++c) {
     const bool more = c + 1 < nchunks;
     CUtensorMap mapH_k;
@@ -606,7 +648,7 @@ fckl_status run(const Request& q) {
       }
       if (more) {
         io = chunk_io(c + 1);
-        if (const fckl_status s1 = stage_in(c + 1, io); s1 != FCKL_OK) return s1;
+        if (const fckl_status s1 = stage_in(c + 1, io, st); s1 != FCKL_OK) return s1;
       }
       continue;
     }
@@ -634,7 +676,7 @@ fckl_status run(const Request& q) {
     if (!bwd) {
       if (more) {
         io = chunk_io(c + 1);
-        if (const fckl_status s1 = stage_in(c + 1, io); s1 != FCKL_OK) return s1;
+        if (const fckl_status s1 = stage_in(c + 1, io, st); s1 != FCKL_OK) return s1;
       }
       continue;
     }
@@ -654,6 +696,14 @@ fckl_status run(const Request& q) {
       ProfScope ps(K_BWD, st, gemm_flops, 2.0 * (io.nr + (double)L.V) * L.H + 2.0 * io.nr * L.V);
       FCKL_LAUNCH((gemm_pair_kernel<EpiDlogits, false, false>), Gv, GEMM_THREADS,
                   pair_smem_bytes<EpiDlogits>(), mapH_k, mapW_k, mapD_st, pb, sa_b, ca);
+    }
+    if (rsd != nullptr && more) {  // next chunk's gather + prep on the second stream
+      const ChunkIO nxt = chunk_io(c + 1);
+      if (cudaEventRecord(rsd->ev[2 * c], st) != cudaSuccess ||
+          cudaStreamWaitEvent(rsd->rs, rsd->ev[2 * c], 0) != cudaSuccess)
+        return FCKL_ERR_CUDA;
+      if (const fckl_status s1 = stage_in(c + 1, nxt, rsd->rs); s1 != FCKL_OK) return s1;
+      if (cudaEventRecord(rsd->ev[2 * c + 1], rsd->rs) != cudaSuccess) return FCKL_ERR_CUDA;
     }
 
     // Backward 2: dH[rows] = alpha * dlogits W; A = dlogits (K-major), B = W (MN-major),
@@ -681,10 +731,15 @@ fckl_status run(const Request& q) {
     }
     const ChunkIO cur = io;
     // The next chunk's gather and teacher prep go ahead of this group's dW
-    // GEMM, so that the next forward GEMM can follow the dW GEMM directly.
+    // GEMM, so that the next forward GEMM can follow the dW GEMM directly
+    // (on the second stream they ran beside this chunk's dH GEMM).
     if (more) {
       io = chunk_io(c + 1);
-      if (const fckl_status s1 = stage_in(c + 1, io); s1 != FCKL_OK) return s1;
+      if (rsd != nullptr) {
+        if (cudaStreamWaitEvent(st, rsd->ev[2 * c + 1], 0) != cudaSuccess) return FCKL_ERR_CUDA;
+      } else if (const fckl_status s1 = stage_in(c + 1, io, st); s1 != FCKL_OK) {
+        return s1;
+      }
     }
 
     // Backward 3, once per group of G chunks (or at the last chunk):

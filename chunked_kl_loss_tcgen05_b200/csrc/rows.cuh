@@ -317,6 +317,12 @@ __global__ void __launch_bounds__(1024)
 // by INT_MAX, which no vocab column matches.  When dH_row0 is given, the warp
 // also zeroes its row of dH (H floats), which the chunk's dH GEMM reduce-adds
 // into.
+// Everything lives in registers (entry k of the row in slot k / 32 of lane
+// k % 32) and warp shuffles; the kernel uses no shared memory, so its blocks fit
+// beside a running GEMM's CTAs.  One pass over the K entries gives each entry
+// its rank in (id, position) order, the summed probability of its id, whether
+// it is the first entry of its id, and the largest id ranked before it (for
+// the tile starts).
 __global__ void __launch_bounds__(ROW_WARPS * 32)
     k_prep_teacher(const int32_t* __restrict__ ids, const float* __restrict__ lg,
                    const uint8_t* __restrict__ mask, RowCount rc, int K, int V, int NT,
@@ -324,9 +330,7 @@ __global__ void __launch_bounds__(ROW_WARPS * 32)
                    float* __restrict__ zs, uint16_t* __restrict__ tstart,
                    float* __restrict__ plogp, DeviceCtl* ctl, float* __restrict__ dH_row0,
                    int H) {
-  __shared__ int s_ids[ROW_WARPS][K_MAX];
-  __shared__ int s_sorted[ROW_WARPS][K_MAX];
-  __shared__ float s_sp[ROW_WARPS][K_MAX];
+  constexpr int S = K_MAX / 32;  // slots per lane
   pdl_wait();
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -337,12 +341,13 @@ __global__ void __launch_bounds__(ROW_WARPS * 32)
     for (int j = lane; j < H / 4; j += 32) z[j] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
   const bool keep = mask == nullptr || mask[row] != 0;
-  float t[K_MAX / 32];
-  int id[K_MAX / 32];
+  const int nslots = (K + 31) / 32;  // warp-uniform
+  float t[S];
+  int id[S];
   float m = -INFINITY;
   bool bad_val = false, bad_id = false;
 #pragma unroll
-  for (int i = 0; i < K_MAX / 32; ++i) {
+  for (int i = 0; i < S; ++i) {
     const int k = lane + 32 * i;
     t[i] = probs ? 0.f : -INFINITY;
     id[i] = INT_MAX;
@@ -358,76 +363,95 @@ __global__ void __launch_bounds__(ROW_WARPS * 32)
       }
       if (d < 0 || d >= V) { bad_id = true; d = INT_MAX; }
       id[i] = d;
-      s_ids[warp][k] = d;
       m = fmaxf(m, t[i]);
     }
   }
   m = warp_max(m);
   bad_val = __any_sync(0xffffffffu, bad_val);
   bad_id = __any_sync(0xffffffffu, bad_id);
-  float p[K_MAX / 32];
+  float p[S];
   if (probs) {
     float s = 0.f;
 #pragma unroll
-    for (int i = 0; i < K_MAX / 32; ++i) s += t[i];
+    for (int i = 0; i < S; ++i) s += t[i];
     s = warp_sum(s);
     if (!(s > 0.f)) bad_val = true;
     const float inv = s > 0.f ? 1.f / s : 0.f;
 #pragma unroll
-    for (int i = 0; i < K_MAX / 32; ++i) p[i] = t[i] * inv;
+    for (int i = 0; i < S; ++i) p[i] = t[i] * inv;
   } else {
     if (!(m > -INFINITY)) bad_val = true;
     const float ms = (m > -INFINITY && m < INFINITY) ? m : 0.f;
     float s = 0.f;
 #pragma unroll
-    for (int i = 0; i < K_MAX / 32; ++i)
+    for (int i = 0; i < S; ++i)
       if (lane + 32 * i < K) s += expf(t[i] - ms);
     s = warp_sum(s);
     const float lse = s > 0.f ? ms + logf(s) : INFINITY;
 #pragma unroll
-    for (int i = 0; i < K_MAX / 32; ++i) p[i] = (lane + 32 * i < K) ? expf(t[i] - lse) : 0.f;
+    for (int i = 0; i < S; ++i) p[i] = (lane + 32 * i < K) ? expf(t[i] - lse) : 0.f;
   }
   if (keep && lane == 0) {
     if (bad_id) atomicOr(&ctl->err, kErrBadIndex);
     if (bad_val) atomicOr(&ctl->err, kErrBadTeacher);
   }
-  __syncwarp();
+  // One pass over the entries j (broadcast slot by slot): for each own entry i,
+  // rank = #{j : (id_j, j) < (id_i, i)}, P = sum of p_j with id_j == id_i,
+  // first = no j < i has id_j == id_i, prev = the largest id_j ranked before i.
+  int rk[S], prev[S];
+  float P[S];
+  bool first[S];
 #pragma unroll
-  for (int i = 0; i < K_MAX / 32; ++i) {
-    const int k = lane + 32 * i;
-    if (k < K) {
-      int rk = 0;
-      for (int j = 0; j < K; ++j) {
-        const int o = s_ids[warp][j];
-        rk += (o < id[i]) || (o == id[i] && j < k);
+  for (int i = 0; i < S; ++i) { rk[i] = 0; prev[i] = -1; P[i] = 0.f; first[i] = true; }
+#pragma unroll
+  for (int js = 0; js < S; ++js) {
+    if (js >= nslots) break;
+    for (int l0 = 0; l0 < 32; l0 += 4) {
+      if (js * 32 + l0 >= K) break;  // warp-uniform
+      int idj[4];
+      float pj[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {  // four independent broadcasts in flight
+        idj[u] = __shfl_sync(0xffffffffu, id[js], l0 + u);
+        pj[u] = __shfl_sync(0xffffffffu, p[js], l0 + u);
       }
-      sid[(size_t)row * K + rk] = id[i];
-      sp[(size_t)row * K + rk] = p[i];
-      zs[(size_t)row * K + rk] = 0.f;
-      s_sorted[warp][rk] = id[i];
-      s_sp[warp][rk] = p[i];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = js * 32 + l0 + u;
+        if (j >= K) break;  // warp-uniform
+#pragma unroll
+        for (int i = 0; i < S; ++i) {
+          if (i >= nslots) break;  // warp-uniform: only the slots that hold entries
+          const int k = lane + 32 * i;
+          const bool before = idj[u] < id[i] || (idj[u] == id[i] && j < k);
+          rk[i] += before ? 1 : 0;
+          prev[i] = before ? max(prev[i], idj[u]) : prev[i];
+          const bool same = idj[u] == id[i];
+          P[i] += same ? pj[u] : 0.f;
+          first[i] = first[i] && !(same && j < k);
+        }
+      }
     }
   }
-  __syncwarp();
-  // sum over distinct ids of P log P, P = the summed probability of an id
   float pl = 0.f;
-  for (int j = lane; j < K; j += 32) {
-    const int idj = s_sorted[warp][j];
-    if (j > 0 && s_sorted[warp][j - 1] == idj) continue;  // not the first entry of its id
-    float P = 0.f;
-    for (int k = j; k < K && s_sorted[warp][k] == idj; ++k) P += s_sp[warp][k];
-    if (P > 0.f) pl += P * logf(P);
+  uint16_t* ts = tstart + (size_t)row * (NT + 1);
+#pragma unroll
+  for (int i = 0; i < S; ++i) {
+    const int k = lane + 32 * i;
+    if (k >= K) continue;
+    sid[(size_t)row * K + rk[i]] = id[i];
+    sp[(size_t)row * K + rk[i]] = p[i];
+    zs[(size_t)row * K + rk[i]] = 0.f;
+    if (first[i] && P[i] > 0.f) pl += P[i] * logf(P[i]);
+    // tiles vt with prev < vt * 256 <= id start at this entry; the last entry
+    // also starts every tile after its own (at K)
+    const long long lo = rk[i] == 0 ? 0 : (long long)prev[i] / BN + 1;
+    const long long hi = min((long long)NT, (long long)id[i] / BN);
+    for (long long vt = lo; vt <= hi; ++vt) ts[vt] = (uint16_t)rk[i];
+    if (rk[i] == K - 1)
+      for (long long vt = (long long)id[i] / BN + 1; vt <= NT; ++vt) ts[vt] = (uint16_t)K;
   }
   pl = warp_sum(pl);
-  for (int vt = lane; vt <= NT; vt += 32) {  // lower bound of vt * 256 in the sorted ids
-    const long long key = (long long)vt * BN;
-    int lo = 0, hi = K;
-    while (lo < hi) {
-      const int mid = (lo + hi) >> 1;
-      if ((long long)s_sorted[warp][mid] < key) lo = mid + 1; else hi = mid;
-    }
-    tstart[(size_t)row * (NT + 1) + vt] = (uint16_t)lo;
-  }
   if (lane == 0) plogp[row] = pl;
 }
 
