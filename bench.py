@@ -47,11 +47,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # launches of one call) from the ncu capture of the current kernels on this workload,
 # summarised under profiles/.  Reset an entry to None when its kernel changes.
 MEASURED_TRAFFIC = {
-    # 256K workload: 2048-row chunks, every launch the same shape as at full size;
-    # captured on a 4096-row cut of it (two chunks), dW = mean over a call's launches
+    # 256K workload: captured on a 4096-row cut of it, whose first chunk (2048
+    # rows) has the full-size launch shape; dW = mean over a full call's launches
     # (one storing launch, the rest reduce-adding)
     "scale_256k_N262144_H4096_V128256_K100_T2": {
-        "fwd_logits_lse": 1.22e9, "bwd_dlogits": 1.77e9, "dH_gemm": 3.65e9, "dW_gemm": 4.68e9},
+        "fwd_logits_lse": 1.24e9, "bwd_dlogits": 1.86e9, "dH_gemm": 3.90e9, "dW_gemm": 4.68e9},
 }
 
 
