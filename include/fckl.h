@@ -37,8 +37,16 @@
  *   - Array pointers are DEVICE pointers into memory the caller owns (except
  *     the host inputs of fckl_fwd_bwd_host).  The library allocates no device
  *     memory; between calls it keeps only a per-device cache of kernel
- *     attributes, the copy stream and events of fckl_fwd_bwd_host, the
+ *     attributes, the copy stream and events of fckl_fwd_bwd_host, a second
+ *     stream and events for the next chunk's row preparation (below), the
  *     profiler's events and the static scratch of fckl_fwd_noalloc.
+ *   - Forward+backward calls of more than one chunk run the next chunk's row
+ *     gather and teacher preparation on that library-owned stream, beside the
+ *     current chunk's dH GEMM; it forks from and joins back into `stream` with
+ *     events, so the call stays ordered on `stream` (and can be captured in a
+ *     CUDA graph from it).  Calls that use it are serialised while they enqueue.
+ *     FCKL_ONE_STREAM=1 in the environment keeps all work on `stream`;
+ *     FCKL_NO_PDL=1 launches the kernels without programmatic dependent launch.
  *   - Arrays are dense and row-major.  hidden, W, dH and dW must start on a
  *     16-byte boundary (TMA), the others on a 4-byte boundary:
  *       hidden     bf16  [N, H]      (raw bfloat16 bit patterns)
