@@ -235,6 +235,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GEMM_THREADS, 1)
   uint32_t* abort_flag = tmem_slot + 1;
   int* split_slot = reinterpret_cast<int*>(abort_flag + 1);
 
+  // A launch over no rows (a chunk past the last compacted row) has no work:
+  // both CTAs of every pair see the same count and leave before setting up
+  // barriers or TMEM (still waiting for the kernel ahead, so that completion
+  // keeps implying the completion of everything before).
+  if (sa.rc.get() <= 0) {
+    pdl_wait();
+    pdl_trigger();
+    return;
+  }
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
