@@ -536,8 +536,8 @@ fckl_status run(const Request& q) {
     const int32_t* ids;
     const float* lg;
     const uint8_t* mask;
-    float* rl;               // row loss of the chunk's first row (out_rows == nullptr)
-    float* dH;               // dH of the chunk's first row (out_rows == nullptr)
+    float* rl;               // row loss of the chunk's first row; with out_rows, of row 0
+    float* dH;               // dH of the chunk's first row; nullptr with out_rows
     const int32_t* out_rows; // gathered rows: the caller's row of each chunk row
     __nv_bfloat16* dlog;     // this chunk's rows in the group's dlogits block
   };
@@ -573,7 +573,8 @@ fckl_status run(const Request& q) {
   };
   // What chunk c needs before its forward GEMM: its host-input piece, its
   // gathered rows (listed and compacted calls) and the teacher preparation
-  // (which also zeroes the chunk's dH rows for the dH GEMM's reduce-adds).
+  // (which, for rows that are not gathered, also zeroes the chunk's dH rows
+  // for the dH GEMM's reduce-adds).
   auto stage_in = [&](long long c, const ChunkIO& io, cudaStream_t ss) -> fckl_status {
     cudaStream_t st = ss;  // the launches below go to this stream
     if (q.ready && cudaStreamWaitEvent(st, q.ready[1 + c], 0) != cudaSuccess) return FCKL_ERR_CUDA;
