@@ -139,7 +139,8 @@ typedef enum { FCKL_TEACHER_LOGITS = 0, FCKL_TEACHER_PROBS = 1 } fckl_teacher_fo
 /* Bytes of device workspace fckl_fwd / fckl_fwd_bwd / fckl_fwd_bwd_rows /
  * fckl_student_entropy need for `prob` (0 when the problem is invalid): the
  * per-chunk teacher and log-sum-exp buffers, the bf16 dlogits of one chunk
- * (of one dW group when dw_rows groups chunks), N floats of row loss, N int32
+ * (of one dW group when dw_rows, or the automatic chunk, groups chunks), two
+ * chunks' staged hidden rows, N floats of row loss, N int32
  * of compacted row list and the staging buffers that row-list and masked
  * calls gather into.  Pure host arithmetic; needs no GPU. */
 size_t fckl_workspace_bytes(const fckl_problem* prob);
