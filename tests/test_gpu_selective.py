@@ -118,3 +118,38 @@ def test_listed_row_out_of_range_is_reported():
     with pytest.raises(FcklError) as ei:
         fused_kl_rows(d[0], d[1], d[2], d[3], rows)
     assert ei.value.status == FCKL_ERR_BAD_INDEX
+
+
+def test_entropy_gptoss_shape_sampled_rows():
+    """Student entropy at the gpt-oss student's H = 2880 and V = 201,088 (a half
+    last vocabulary tile) on 64 sampled rows of a 1024-row batch."""
+    inp = synth.make_custom(1024, 2880, 201088, 4, T=1.0, mask_frac=0.03, seed=1003)
+    rows = synth.sample_rows(inp, 64)
+    d = arrays_to_device(inp.hidden, inp.W, inp.topk_idx, inp.topk_logit, inp.row_mask)
+    e = student_entropy(d[0], d[1], d[4], T=1.0).cpu().numpy()
+    _, ref = oracle.student_entropy(inp.hidden, inp.W, 1.0, inp.row_mask, rows=rows)
+    np.testing.assert_allclose(e[rows], ref, rtol=RTOL, atol=1e-4)
+    assert (e[inp.row_mask == 0] == 0).all()
+
+
+@pytest.mark.parametrize("chunk,dw_rows", [(0, 0), (48, 96)])
+def test_listed_rows_with_sampled_targets(chunk, dw_rows):
+    """The listed-row entry point with RS-KD sampled class weights (repeated ids)
+    against the oracle's "probs" teacher over the same rows."""
+    N, H, V, K, T = 600, 192, 3000, 24, 1.5
+    inp = synth.make_sampled_targets(N, H, V, K, T=T, seed=77)
+    rng = np.random.default_rng(77)
+    rows = np.sort(rng.choice(N, 150, replace=False))
+    d = arrays_to_device(inp.hidden, inp.W, inp.topk_idx, inp.topk_logit, None)
+    loss, rl, dH, dW = fused_kl_rows(d[0], d[1], d[2], d[3],
+                                     torch.from_numpy(rows.astype(np.int32)).cuda(), T=T,
+                                     chunk=chunk, dw_rows=dw_rows, want_row_loss=True, teacher=1)
+    torch.cuda.synchronize()
+    mask = np.zeros(N, np.uint8)
+    mask[rows] = 1
+    o = oracle.fused_chunked_kl(inp.hidden, inp.W, inp.topk_idx, inp.topk_logit, mask, T,
+                                teacher="probs")
+    assert abs(loss.item() - o["loss"]) <= RTOL * abs(o["loss"])
+    np.testing.assert_allclose(rl.cpu().numpy(), o["row_loss"], rtol=RTOL, atol=1e-4)
+    assert rel_fro(dH.cpu().numpy(), o["dH"]) <= GRAD_RTOL
+    assert rel_fro(dW.cpu().numpy(), o["dW"]) <= GRAD_RTOL
