@@ -88,6 +88,8 @@ def parse():
     ap.add_argument("--graph", action="store_true",
                     help="also time the step replayed from a captured CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-grouped", action="store_true",
+                    help="skip the extra timing with chunks grouped per dW GEMM (dw_grouped)")
     ap.add_argument("--cpu-rows", type=int, default=0, help="rows in the oracle sample (0 = auto)")
     ap.add_argument("--profile-json", default="")
     ap.add_argument("--mem-sweep", action="store_true",
@@ -388,6 +390,14 @@ def run_cuda(args):
     if args.graph and mode != "dp":
         graph = measure_graph(torch, dev, step, args.steps, cfg, world)
 
+    # A workload whose explicit chunk is below 4096 rows also runs with chunks
+    # grouped so that each dW GEMM covers >= 4096 rows (fckl_problem.dw_rows):
+    # the speed the library's memory/speed knob buys back, same box, same inputs.
+    grouped = None
+    if (not args.no_grouped and mode == "single" and args.dw_rows == 0 and 0 < C < 4096
+            and cfg.N > C):
+        grouped = measure_grouped(torch, dev, d, cfg, args.steps, outs, flops_step, burst)
+
     e2e = None
     if not args.no_e2e:
         if mode == "dp":
@@ -421,6 +431,7 @@ def run_cuda(args):
                 "peak_mem_gib": peak_gib, "loss": loss_val,
                 "roofline": roofline, "kernels": kernels,
                 "cpu_baseline": cpu, "e2e": e2e, "clocks": clk, "graph": graph,
+                "dw_grouped": grouped,
                 "gpu_launches": launches_per_step * args.steps}
         print(json.dumps(line), flush=True)
         if args.profile_json:
@@ -430,6 +441,45 @@ def run_cuda(args):
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def measure_grouped(torch, dev, d, cfg, steps, outs, flops_step, burst):
+    """The same workload with dw_rows = 4096 (two or more chunks per dW GEMM; the
+    workspace then holds that many rows of dlogits): step time and the dW GEMM's
+    rate, its launches event-timed in the last quarter of the steps."""
+    from chunked_kl_loss_tcgen05_b200 import (FcklProblem, fckl_profile_begin, fckl_profile_end,
+                                              fckl_workspace_bytes)
+    from chunked_kl_loss_tcgen05_b200.torch_api import alloc_workspace, fused_kl_fwd_bwd
+    prob = FcklProblem(cfg.N, cfg.H, cfg.V, cfg.K, cfg.T, cfg.chunk, dw_rows=4096)
+    ws = alloc_workspace(prob, dev)
+
+    def step():
+        return fused_kl_fwd_bwd(*d, T=cfg.T, chunk=cfg.chunk, workspace=ws, check=False, out=outs,
+                                dw_rows=4096)
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_prof = max(1, min(steps, max(2, steps // 4)))
+    e0.record(stream)
+    for i in range(steps):
+        if i == steps - n_prof:
+            fckl_profile_begin(["dW_gemm"])
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    prof = fckl_profile_end()
+    ms = e0.elapsed_time(e1) / steps
+    dw = next((p for p in prof if p["name"] == "dW_gemm"), None)
+    dw_tflops = dw["flops"] / (dw["total_ms"] / 1e3) / 1e12 if dw and dw["total_ms"] > 0 else None
+    out = {"dw_rows": 4096, "ms_per_step": ms, "value": cfg.N / (ms / 1e3), "unit": "tokens/s",
+           "tflops": flops_step / (ms / 1e3) / 1e12, "frac_of_burst": flops_step / (ms / 1e3) / 1e12 / burst,
+           "dW_gemm_tflops": dw_tflops, "steps": steps,
+           "workspace_gib": fckl_workspace_bytes(prob) / 2**30}
+    del ws
+    torch.cuda.empty_cache()
+    return out
 
 
 def max_over_ranks(torch, dev, ms, world):
