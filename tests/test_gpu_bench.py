@@ -40,3 +40,19 @@ def test_bench_contract_line(mode):
         assert d["config"]["parallelism"].startswith("dp1")
     else:
         assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] > 0
+
+
+def test_memory_sweep_is_linear_in_rows():
+    """bench.py --mem-sweep: peak device memory of one forward+backward call grows
+    by the per-row inputs and outputs only (hidden 8 KiB, dH 16 KiB, teacher
+    0.78 KiB, two per-row words), and an explicit chunk bounds the rest."""
+    r = subprocess.run([sys.executable, "bench.py", "--mem-sweep", "--sweep-chunk", "256",
+                        "--sweep-s", "1024,2048,4096"], cwd=ROOT, capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    d = json.loads(r.stdout.strip().splitlines()[-1])
+    per_row_kib = (4096 * 2 + 4096 * 4 + 100 * 8 + 8) / 1024
+    assert abs(d["fit"]["slope_kib_per_row"] - per_row_kib) < 0.05
+    assert d["fit"]["r2"] > 0.9999
+    # W (1 GiB) + dW (2 GiB) + one 256-row chunk of dlogits and per-chunk buffers
+    assert 2.9 < d["fit"]["intercept_gib"] < 3.1
