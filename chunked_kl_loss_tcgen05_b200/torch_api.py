@@ -44,15 +44,69 @@ def alloc_workspace(prob: FcklProblem, device) -> torch.Tensor:
     return torch.empty(nbytes, dtype=torch.uint8, device=device)
 
 
+def _check_shapes(hidden, W, topk_idx=None, topk_logit=None, row_mask=None):
+    """Shapes and dtypes the library reads without further checks: hidden [N,H],
+    W [V,H], topk_idx int32 and topk_logit float32 [N,K], row_mask uint8 [N]."""
+    if hidden.dim() != 2 or W.dim() != 2 or W.shape[1] != hidden.shape[1]:
+        raise ValueError(f"hidden must be [N,H] and W [V,H]; got {tuple(hidden.shape)} "
+                         f"and {tuple(W.shape)}")
+    N = hidden.shape[0]
+    if topk_idx is not None:
+        if (topk_idx.dim() != 2 or tuple(topk_logit.shape) != tuple(topk_idx.shape)
+                or topk_idx.shape[0] != N):
+            raise ValueError(f"topk_idx and topk_logit must both be [N={N},K]; got "
+                             f"{tuple(topk_idx.shape)} and {tuple(topk_logit.shape)}")
+        if topk_idx.dtype != torch.int32 or topk_logit.dtype != torch.float32:
+            raise TypeError("topk_idx must be int32 and topk_logit float32")
+    if row_mask is not None:
+        if row_mask.dtype != torch.uint8 or row_mask.numel() != N:
+            raise TypeError(f"row_mask must be a uint8 tensor of N={N} entries")
+
+
+def _check_placement(cuda, tensors):
+    """Every named tensor contiguous and on one CUDA device (cuda=True) or on
+    the host (cuda=False)."""
+    devices = set()
+    for name, t in tensors:
+        if t is None:
+            continue
+        where = "CUDA" if cuda else "CPU"
+        if t.is_cuda != cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous {where} tensor")
+        devices.add(t.device)
+    if cuda and len(devices) > 1:
+        raise ValueError(f"all tensors must be on one device; got {sorted(map(str, devices))}")
+
+
+def _workspace(workspace, prob, device, host_inputs=False):
+    """The caller's workspace (a contiguous uint8 tensor on ``device``; the
+    library checks its size), or a new one of the size the problem needs."""
+    if workspace is None:
+        return (alloc_host_workspace if host_inputs else alloc_workspace)(prob, device)
+    if workspace.dtype != torch.uint8 or not workspace.is_contiguous() or workspace.device != device:
+        raise ValueError(f"workspace must be a contiguous uint8 tensor on {device}")
+    return workspace
+
+
+def _check_out(out, prob, device, with_loss=True):
+    """Caller-supplied outputs: (loss[>=1],) dH [N,H], dW [V,H], contiguous float32
+    tensors on the inputs' device."""
+    names = ("loss", "dH", "dW") if with_loss else ("dH", "dW")
+    if len(out) != len(names):
+        raise ValueError("out must be (" + ", ".join(names) + ")")
+    want = {"loss": None, "dH": (prob.N, prob.H), "dW": (prob.V, prob.H)}
+    for name, t in zip(names, out):
+        shape_ok = t.numel() >= 1 if want[name] is None else tuple(t.shape) == want[name]
+        if (not shape_ok or t.dtype != torch.float32 or not t.is_contiguous()
+                or t.device != device):
+            raise ValueError(f"out {name} must be a contiguous float32 tensor on {device}"
+                             + ("" if want[name] is None else f" of shape {want[name]}"))
+
+
 def _check_inputs(hidden, W, topk_idx, topk_logit, row_mask):
-    for name, t in (("hidden", hidden), ("W", W), ("topk_idx", topk_idx),
-                    ("topk_logit", topk_logit)):
-        if not t.is_cuda or not t.is_contiguous():
-            raise ValueError(f"{name} must be a contiguous CUDA tensor")
-    if topk_idx.dtype != torch.int32 or topk_logit.dtype != torch.float32:
-        raise TypeError("topk_idx must be int32 and topk_logit float32")
-    if row_mask is not None and (row_mask.dtype != torch.uint8 or not row_mask.is_contiguous()):
-        raise TypeError("row_mask must be a contiguous uint8 tensor")
+    _check_shapes(hidden, W, topk_idx, topk_logit, row_mask)
+    _check_placement(True, (("hidden", hidden), ("W", W), ("topk_idx", topk_idx),
+                            ("topk_logit", topk_logit), ("row_mask", row_mask)))
 
 
 def fused_kl_fwd_bwd(hidden, W, topk_idx, topk_logit, row_mask=None, T=1.0, chunk=0,
@@ -69,14 +123,10 @@ def fused_kl_fwd_bwd(hidden, W, topk_idx, topk_logit, row_mask=None, T=1.0, chun
     _check_inputs(hidden, W, topk_idx, topk_logit, row_mask)
     prob = make_problem(hidden, W, topk_idx, T, chunk, teacher, n_valid_total, dw_rows)
     dev = hidden.device
-    if workspace is None:
-        workspace = alloc_workspace(prob, dev)
+    workspace = _workspace(workspace, prob, dev)
     if out is not None:
+        _check_out(out, prob, dev)
         loss, dH, dW = out
-        if (loss.numel() < 1 or tuple(dH.shape) != (prob.N, prob.H)
-                or tuple(dW.shape) != (prob.V, prob.H) or dH.dtype != torch.float32
-                or dW.dtype != torch.float32 or not dH.is_contiguous() or not dW.is_contiguous()):
-            raise ValueError("out must be (loss[>=1], dH[N,H], dW[V,H]) contiguous float32")
     else:
         loss = torch.empty(1, dtype=torch.float32, device=dev)
         dH = torch.empty(prob.N, prob.H, dtype=torch.float32, device=dev)
@@ -108,12 +158,12 @@ def fused_kl_fwd_bwd_sliced(hidden, W, topk_idx, topk_logit, row_mask=None, T=1.
     _check_inputs(hidden, W, topk_idx, topk_logit, row_mask)
     prob = make_problem(hidden, W, topk_idx, T, chunk, teacher, n_valid_total, dw_rows)
     dev = hidden.device
-    if workspace is None:
-        workspace = alloc_workspace(prob, dev)
+    workspace = _workspace(workspace, prob, dev)
     if out is None:
         out = (torch.empty(1, dtype=torch.float32, device=dev),
                torch.empty(prob.N, prob.H, dtype=torch.float32, device=dev),
                torch.empty(prob.V, prob.H, dtype=torch.float32, device=dev))
+    _check_out(out, prob, dev)
     loss, dH, dW = out
     stream = torch.cuda.current_stream(dev)
     events = [torch.cuda.Event() for _ in range(n_slices)]
@@ -138,8 +188,7 @@ def fused_kl_fwd(hidden, W, topk_idx, topk_logit, row_mask=None, T=1.0, chunk=0,
     _check_inputs(hidden, W, topk_idx, topk_logit, row_mask)
     prob = make_problem(hidden, W, topk_idx, T, chunk, teacher)
     dev = hidden.device
-    if workspace is None:
-        workspace = alloc_workspace(prob, dev)
+    workspace = _workspace(workspace, prob, dev)
     loss = torch.empty(1, dtype=torch.float32, device=dev)
     row_loss = torch.empty(prob.N, dtype=torch.float32, device=dev) if want_row_loss else None
     stream = torch.cuda.current_stream(dev).cuda_stream
@@ -172,23 +221,17 @@ def fused_kl_fwd_bwd_host(hidden, W, topk_idx, topk_logit, row_mask=None, T=1.0,
     the kernels.  Returns (loss as a Python float, dH, dW); the loss read
     synchronises the stream."""
     hidden, W = _bits(hidden), _bits(W)
-    for name, t in (("hidden", hidden), ("topk_idx", topk_idx), ("topk_logit", topk_logit)):
-        if t.is_cuda or not t.is_contiguous():
-            raise ValueError(f"{name} must be a contiguous CPU tensor")
-    if row_mask is not None and (row_mask.is_cuda or row_mask.dtype != torch.uint8
-                                 or not row_mask.is_contiguous()):
-        raise TypeError("row_mask must be a contiguous uint8 CPU tensor")
-    if not W.is_cuda or not W.is_contiguous():
-        raise ValueError("W must be a contiguous CUDA tensor")
-    if topk_idx.dtype != torch.int32 or topk_logit.dtype != torch.float32:
-        raise TypeError("topk_idx must be int32 and topk_logit float32")
+    _check_shapes(hidden, W, topk_idx, topk_logit, row_mask)
+    _check_placement(False, (("hidden", hidden), ("topk_idx", topk_idx),
+                             ("topk_logit", topk_logit), ("row_mask", row_mask)))
+    _check_placement(True, (("W", W),))
     prob = make_problem(hidden, W, topk_idx, T, chunk, dw_rows=dw_rows)
     dev = W.device
-    if workspace is None:
-        workspace = alloc_host_workspace(prob, dev)
+    workspace = _workspace(workspace, prob, dev, host_inputs=True)
     if out is None:
         out = (torch.empty(prob.N, prob.H, dtype=torch.float32, device=dev),
                torch.empty(prob.V, prob.H, dtype=torch.float32, device=dev))
+    _check_out(out, prob, dev, with_loss=False)
     dH, dW = out
     if loss_host is None:
         loss_host = torch.empty(1, dtype=torch.float32, pin_memory=True)
@@ -267,11 +310,12 @@ def student_entropy(hidden, W, row_mask=None, T=1.0, chunk=0, workspace=None, ch
     """Per-row student entropy H(softmax(W h / T)) in nats, [N] fp32 (0 for masked rows)."""
     from . import fckl_student_entropy
     hidden, W = _bits(hidden), _bits(W)
+    _check_shapes(hidden, W, row_mask=row_mask)
+    _check_placement(True, (("hidden", hidden), ("W", W), ("row_mask", row_mask)))
     N, H = hidden.shape
     prob = FcklProblem(N, H, W.shape[0], 1, T, chunk)
     dev = hidden.device
-    if workspace is None:
-        workspace = alloc_workspace(prob, dev)
+    workspace = _workspace(workspace, prob, dev)
     ent = torch.empty(N, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev).cuda_stream
     st = fckl_student_entropy(prob, hidden.data_ptr(), W.data_ptr(),
@@ -289,6 +333,11 @@ def student_entropy(hidden, W, row_mask=None, T=1.0, chunk=0, workspace=None, ch
 def select_top_rows(score, n_select, row_mask=None):
     """(rows int32 [n_select] ascending, padded with -1; count int32 [1]) on device."""
     from . import fckl_select_top_rows
+    if score.dtype != torch.float32 or score.dim() != 1:
+        raise TypeError("score must be a 1-D float32 tensor")
+    if row_mask is not None and (row_mask.dtype != torch.uint8 or row_mask.numel() != score.numel()):
+        raise TypeError("row_mask must be a uint8 tensor with one entry per score")
+    _check_placement(True, (("score", score), ("row_mask", row_mask)))
     N = score.numel()
     rows = torch.empty(n_select, dtype=torch.int32, device=score.device)
     count = torch.empty(1, dtype=torch.int32, device=score.device)
@@ -305,11 +354,13 @@ def fused_kl_rows(hidden, W, topk_idx, topk_logit, rows, T=1.0, chunk=0, workspa
     """Loss (and dH, dW) over the listed rows only.  Returns (loss, row_loss, dH, dW)."""
     from . import fckl_fwd_bwd_rows
     hidden, W = _bits(hidden), _bits(W)
+    if rows.dtype != torch.int32 or rows.dim() != 1:
+        raise TypeError("rows must be a 1-D int32 tensor")
     _check_inputs(hidden, W, topk_idx, topk_logit, None)
+    _check_placement(True, (("hidden", hidden), ("rows", rows)))
     prob = make_problem(hidden, W, topk_idx, T, chunk, teacher, dw_rows=dw_rows)
     dev = hidden.device
-    if workspace is None:
-        workspace = alloc_workspace(prob, dev)
+    workspace = _workspace(workspace, prob, dev)
     loss = torch.empty(1, dtype=torch.float32, device=dev)
     row_loss = torch.empty(prob.N, dtype=torch.float32, device=dev) if want_row_loss else None
     dH = torch.empty(prob.N, prob.H, dtype=torch.float32, device=dev) if grads else None
