@@ -58,6 +58,9 @@
  *       row_loss   fp32  [N] or NULL (per-row l_r, 0 for masked rows)
  *       dH         fp32  [N, H]      overwritten
  *       dW         fp32  [V, H]      overwritten
+ *     A pointer carries no length: each array must hold the elements listed
+ *     (a shorter buffer is read or written past its end).  The PyTorch helpers
+ *     of the binding check tensor shapes before they call the library.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
  *     asynchronous on that stream; the workspace must not be shared by calls
  *     that can overlap.
